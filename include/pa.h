@@ -1,0 +1,219 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged-KV attention for continuous batching on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three pages on continuous batching and
+ * PagedAttention:
+ *   [CB]  "Continuous batching and PagedAttention" (how-ai-works, chapter 7)
+ *   [PS]  "Production Serving: Continuous Batching and PagedAttention"
+ *         (llm-under-the-hood, project 17)
+ *   [TR]  "Continuous batching and PagedAttention: serving many users from
+ *         one GPU" (trefon.com notes)
+ *
+ * ---------------------------------------------------------------- layout --
+ * KV cache: two device arrays, k_cache and v_cache, each
+ *     [num_blocks][num_kv_heads][PA_BLOCK_SIZE = 16][head_dim]
+ * row-major, element type bf16 or fp8 E4M3 (OCP "fn" variant).  Physical
+ * block p of kv head h is one contiguous run of 16*head_dim elements
+ * ([PS] "PagedAttention, the thing you build for memory": fixed 16-token
+ * pages in one pre-allocated pool; [TR] "Fragmentation: PagedAttention").
+ * The pages print two contradictory interleaved K/V layouts; this library
+ * keeps K and V in separate arrays.
+ *
+ * Block table: int32 [num_seqs][max_blocks_per_seq]; entry [b][j] is the
+ * physical block holding logical tokens 16j..16j+15 of sequence b ([PS]
+ * Step 4 "Implement the paged KV cache": page table, logical block ->
+ * physical page).  Entries at or past ceil(seq_len/16) are never read.
+ *
+ * Slot mapping: int64 [num_tokens]; slot = physical_block*16 + offset.
+ * A negative slot marks a padding token that is skipped.
+ *
+ * Grouped-query attention: query head h reads kv head
+ * floor(h * num_kv_heads / num_q_heads) (consecutive query heads share one
+ * kv head).
+ *
+ * fp8 cache: one fp32 scale per kv head for K and one for V.  A stored code
+ * c means the value e4m3(c) * scale[h].  Writing encodes
+ *     c = e4m3_rn_satfinite(x * rn(1/scale[h]))
+ * -- one IEEE fp32 multiply by the correctly rounded fp32 reciprocal, then
+ * round-to-nearest-even to E4M3 with finite overflow and infinities clamped
+ * to +-448.
+ *
+ * -------------------------------------------------------- conventions --
+ * All array arguments are DEVICE pointers on the current device unless
+ * stated otherwise.  The caller owns every buffer and the stream; the
+ * library never allocates or frees memory and never synchronises, except
+ * pa_get_last_device_error(), which reads a status word back.  Every call
+ * enqueues its kernels on `stream` (a cudaStream_t; NULL = legacy default
+ * stream) and returns at once.
+ *
+ * Every entry point returns a pa_status.  Argument errors are detected on
+ * the host before anything is enqueued.  Metadata read on the device (block
+ * ids, slots, lengths) is bounds-checked by the kernels: an out-of-range
+ * value is skipped (treated as absent) and recorded in the device status
+ * word, which pa_get_last_device_error() returns.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_BLOCK_SIZE 16
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = -1, /* null pointer, bad size, Hq % Hkv != 0, block_size != 16 */
+    PA_ERR_UNSUPPORTED = -2, /* valid but not built: head_dim not in {64,128}, group > 8, ... */
+    PA_ERR_WORKSPACE = -3,   /* workspace missing or smaller than pa_decode_workspace_size() */
+    PA_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+    PA_ERR_DEVICE = -5,      /* returned by pa_get_last_device_error when a kernel flagged bad metadata */
+    PA_ERR_TIMEOUT = -6      /* reserved for host-side waits; device waits report PA_DEVERR_TIMEOUT */
+} pa_status;
+
+typedef enum pa_dtype {
+    PA_DTYPE_BF16 = 0,
+    PA_DTYPE_FP8_E4M3 = 1
+} pa_dtype;
+
+/* Bits of the device status word (pa_get_last_device_error). */
+#define PA_DEVERR_BAD_BLOCK 0x1u  /* a block-table entry outside [0, num_blocks) was needed */
+#define PA_DEVERR_BAD_SLOT 0x2u   /* a slot mapped past the last block */
+#define PA_DEVERR_BAD_LEN 0x4u    /* seq_len < 0 or > 16 * max_blocks_per_seq */
+#define PA_DEVERR_BAD_PAIR 0x8u   /* a copy pair outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait for an async copy or MMA gave up (results invalid) */
+
+/* An opaque stream handle: pass a cudaStream_t. */
+typedef void *pa_stream_t;
+
+/* Shape of the paged cache.  block_size must be 16; head_dim 64 or 128;
+ * dtype a pa_dtype. */
+typedef struct pa_cache_desc {
+    int64_t num_blocks;
+    int32_t num_kv_heads;
+    int32_t block_size;
+    int32_t head_dim;
+    int32_t dtype;
+} pa_cache_desc;
+
+/*
+ * pa_write_kv -- slot-mapped write of new K/V ("reshape_and_cache").
+ * [PS] Step 4 "Implement the paged KV cache": each new token's K and V land
+ * in slot (length mod 16) of the sequence's current page; here the host
+ * allocator has already turned that into one slot per token.
+ *
+ *   k, v          bf16 [num_tokens][num_kv_heads][head_dim], contiguous.
+ *   slot_mapping  int64 [num_tokens]; slot < 0 skips the token.
+ *   k_cache, v_cache  the cache (layout above), written in place.
+ *   k_scale, v_scale  fp32 [num_kv_heads]; required for an fp8 cache,
+ *                 ignored (may be NULL) for bf16.
+ * For bf16 the cache receives the input bits unchanged.  Tokens must map to
+ * distinct slots (otherwise which write wins is unspecified).
+ * num_tokens == 0 enqueues nothing.
+ */
+int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping, int64_t num_tokens, void *k_cache,
+                void *v_cache, const float *k_scale, const float *v_scale, const pa_cache_desc *desc,
+                pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copy.
+ * [CB] "PagedAttention: KV cache memory": blocks shared with copy-on-write
+ * are copied when a sharer diverges; [TR] "Fragmentation: PagedAttention":
+ * sequences with a common prefix point at the same blocks until they
+ * diverge.
+ *
+ *   src_dst_pairs  int32 [num_pairs][2] = (src, dst) physical block ids.
+ * Every element of block src (all kv heads, all 16 slots) is copied to block
+ * dst in both caches.  Destinations must be distinct and no destination may
+ * also be a source in the same call (pairs run concurrently).
+ * Per-head fp8 scales are per cache, not per block: nothing else to copy.
+ * num_pairs == 0 enqueues nothing.
+ */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, int32_t num_pairs,
+                   const pa_cache_desc *desc, pa_stream_t stream);
+
+/*
+ * pa_decode_workspace_size -- bytes of device workspace pa_decode needs for
+ * this shape (host function, no device work).  partition_tokens as for
+ * pa_decode.
+ */
+int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+                             int32_t partition_tokens, size_t *bytes);
+
+/*
+ * pa_decode -- paged decode attention, one query token per sequence.
+ * [PS] Step 6 "Implement attention over paged storage", per query head:
+ *     out[b][h] = sum_{t < seq_lens[b]} softmax_t(scale * q[b][h] . k_t) * v_t
+ * with k_t, v_t stored at slot t%16 of block block_tables[b][t/16], kv head
+ * floor(h*Hkv/Hq).  The sequence's own newest token must already be in the
+ * cache (write first, then attend).
+ *
+ *   out           bf16 [num_seqs][num_q_heads][head_dim] (fp32 accumulation,
+ *                 rounded to nearest-even bf16 once at the end).
+ *   q             bf16 [num_seqs][num_q_heads][head_dim].
+ *   block_tables  int32 [num_seqs][max_blocks_per_seq].
+ *   seq_lens      int32 [num_seqs]; 0 gives an all-zero output row.
+ *   scale         softmax scale (typically 1/sqrt(head_dim)).
+ *   k_scale, v_scale  fp32 [num_kv_heads] for an fp8 cache, else ignored.
+ *   partition_tokens  split-K partition length in tokens: a multiple of 16
+ *                 in [16, 4096], or 0 for the library default (256).  Each
+ *                 partition of a sequence yields a partial result and its
+ *                 log-sum-exp; sequences with more than one partition are
+ *                 combined by a log-sum-exp merge.  Partition boundaries
+ *                 depend only on the token index, so a sequence's result
+ *                 does not depend on the rest of the batch.
+ *   workspace     device scratch of at least pa_decode_workspace_size()
+ *                 bytes, 256-byte aligned; contents need no initialisation
+ *                 and are garbage afterwards.
+ * num_seqs must be in [1, 2048]; num_q_heads / num_kv_heads in {1,2,4,8}.
+ */
+int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
+              const int32_t *seq_lens, int32_t num_seqs, int32_t max_blocks_per_seq, int32_t num_q_heads,
+              float scale, const float *k_scale, const float *v_scale, int32_t partition_tokens,
+              void *workspace, size_t workspace_bytes, const pa_cache_desc *desc, pa_stream_t stream);
+
+/*
+ * pa_prefill_chunk -- causal attention of prompt chunks over their paged
+ * prefixes (chunked prefill).
+ * [CB] "How the scheduler works": a long prompt is cut into chunks that fit
+ * the per-step token budget; [TR] "Prefill gets in the way": chunks are
+ * interleaved with decode steps.
+ *
+ *   out, q        bf16 [total_q][num_q_heads][head_dim].
+ *   cu_q_lens     int32 [num_chunks+1]: chunk c owns rows
+ *                 cu_q_lens[c]..cu_q_lens[c+1]-1.
+ *   prefix_lens   int32 [num_chunks]: tokens already in the cache before the
+ *                 chunk.  Row i of chunk c sits at position prefix_lens[c]+i
+ *                 and attends keys 0..prefix_lens[c]+i inclusive.
+ *   block_tables  int32 [num_chunks][max_blocks_per_seq].
+ *   max_q_len     host upper bound on any chunk's length (sizes the grid).
+ * The chunk's own K/V must already be in the cache (pa_write_kv first).
+ * bf16 cache only; an fp8 cache returns PA_ERR_UNSUPPORTED.
+ */
+int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const int32_t *prefix_lens,
+                     const int32_t *block_tables, int32_t num_chunks, int32_t max_blocks_per_seq,
+                     int32_t num_q_heads, int32_t max_q_len, const void *k_cache, const void *v_cache, float scale,
+                     const float *k_scale, const float *v_scale, const pa_cache_desc *desc, pa_stream_t stream);
+
+/*
+ * pa_get_last_device_error -- synchronise `stream`, return the device status
+ * word (PA_DEVERR_* bits, 0 if clean) in *flags and clear it.  Returns
+ * PA_ERR_DEVICE if any bit was set, PA_OK otherwise.
+ */
+int pa_get_last_device_error(uint32_t *flags, pa_stream_t stream);
+
+/* Human-readable name of a pa_status value (static string). */
+const char *pa_status_string(int status);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

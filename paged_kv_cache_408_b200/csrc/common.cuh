@@ -1,0 +1,121 @@
+// common.cuh -- small sm_100a device helpers shared by the libpa kernels:
+// mbarriers, 1-D bulk async copies (the TMA engine's untiled form), packed
+// fp32x2 FMA, bf16 / fp8 unpacking and the base-2 exponential.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+#define PA_DEVICE __device__ __forceinline__
+
+namespace pa {
+
+// ------------------------------------------------------------------ mbarrier
+PA_DEVICE uint32_t smem_addr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+PA_DEVICE void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+PA_DEVICE void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+// Arrive on `bar` and add `bytes` to the transaction count it waits for.
+PA_DEVICE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+PA_DEVICE void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+PA_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+PA_DEVICE uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for phase `parity` of `bar` to complete.  The wait is bounded: after
+// about `limit_ns` nanoseconds it gives up and returns false, so a lost
+// transaction can never hang the GPU; the caller records PA_DEVERR_TIMEOUT.
+PA_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > limit_ns) return false;
+    return true;
+}
+
+// ------------------------------------------------------- 1-D bulk async copy
+// Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte
+// aligned) completing on `bar` as a transaction.  No multicast.
+PA_DEVICE void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ----------------------------------------------------------------- arithmetic
+// Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, lane-wise, RN.
+PA_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(reinterpret_cast<unsigned long long &>(d))
+        : "l"(reinterpret_cast<unsigned long long &>(a)), "l"(reinterpret_cast<unsigned long long &>(b)),
+          "l"(reinterpret_cast<unsigned long long &>(c)));
+    return d;
+}
+
+PA_DEVICE float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(reinterpret_cast<unsigned long long &>(d))
+        : "l"(reinterpret_cast<unsigned long long &>(a)), "l"(reinterpret_cast<unsigned long long &>(b)));
+    return d;
+}
+
+// 2^x with the hardware approximation (MUFU.EX2), flushing denormal results.
+PA_DEVICE float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Two bf16 packed in one 32-bit word -> (low element, high element) as fp32.
+// bf16 is the upper half of a binary32, so widening is a shift / mask.
+PA_DEVICE float2 bf16x2_to_float2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// Two E4M3 codes packed in 16 bits (low byte first) -> fp32 pair.
+PA_DEVICE float2 e4m3x2_to_float2(uint16_t w) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
+    return __half22float2(*reinterpret_cast<__half2 *>(&h));
+}
+
+// Device status word (PA_DEVERR_* bits).
+PA_DEVICE void flag_error(unsigned *err, unsigned bits) {
+    if (err) atomicOr(err, bits);
+}
+
+}  // namespace pa

@@ -1,0 +1,104 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+include/pa.h declares, and rejects bad arguments on the host before any
+device work (no compute call is made here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_408_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = C.c_void_p(0x10000)  # never dereferenced: every call below fails validation first
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    fns = header_functions()
+    for f in ("pa_write_kv", "pa_decode", "pa_decode_workspace_size", "pa_prefill_chunk", "pa_copy_blocks",
+              "pa_get_last_device_error", "pa_status_string"):
+        assert f in fns
+
+
+def test_library_exports_every_declared_symbol():
+    L = ops.lib()
+    for f in header_functions():
+        assert hasattr(L, f), f
+
+
+def test_status_strings_and_version():
+    assert ops.status_string(0) == "PA_OK"
+    assert ops.status_string(-1) == "PA_ERR_INVALID_ARG"
+    assert ops.status_string(-3) == "PA_ERR_WORKSPACE"
+    assert ops.lib().pa_version() >= 100
+
+
+def desc(nb=64, hkv=8, bs=16, d=128, dt=0):
+    return ops.CacheDesc(nb, hkv, bs, d, dt)
+
+
+def call_decode(d, B=4, maxb=8, Hq=32, part=0, ws=None, ws_bytes=0, ptr=FAKE):
+    return ops.lib().pa_decode(ptr, ptr, ptr, ptr, ptr, ptr, B, maxb, Hq, 0.1, ptr, ptr, part, ws, ws_bytes,
+                               C.byref(d) if d is not None else None, None)
+
+
+def test_decode_rejects_bad_arguments_on_host():
+    assert call_decode(None) == -1
+    assert call_decode(desc(bs=8)) == -1
+    assert call_decode(desc(d=96)) == -2
+    assert call_decode(desc(dt=7)) == -1
+    assert call_decode(desc(), Hq=30) == -1          # Hq % Hkv != 0
+    assert call_decode(desc(hkv=2), Hq=32) == -2     # group of 16 not built
+    assert call_decode(desc(), B=5000) == -1
+    assert call_decode(desc(), part=20) == -1        # not a multiple of 16
+    assert call_decode(desc(), part=4096) == -1      # above the largest partition
+    assert call_decode(desc(), ptr=None) == -1       # null pointers
+    # several partitions need a workspace of the reported size
+    assert call_decode(desc(), maxb=64, part=256) == -3
+    assert call_decode(desc(), B=0) == 0             # nothing to do
+
+
+def test_workspace_size():
+    assert ops.decode_workspace_size(64, 32, 128, 16, 256) == 0  # one partition: no workspace
+    n = ops.decode_workspace_size(64, 32, 128, 128, 256)          # 2048 tokens -> 8 partitions
+    assert n >= 64 * 32 * 8 * (128 + 1) * 4
+    assert ops.decode_workspace_size(64, 32, 128, 128, 512) < n
+    with pytest.raises(ops.PAError):
+        ops.decode_workspace_size(64, 32, 96, 128)
+
+
+def test_write_and_copy_reject_bad_arguments_on_host():
+    L = ops.lib()
+    d = desc()
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, None, C.byref(desc(d=80)), None) == -2
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, -1, FAKE, FAKE, None, None, C.byref(d), None) == -1
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 0, FAKE, FAKE, None, None, C.byref(d), None) == 0
+    assert L.pa_write_kv(FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, None, C.byref(desc(dt=1)), None) == -1  # fp8 needs scales
+    assert L.pa_write_kv(None, FAKE, FAKE, 4, FAKE, FAKE, None, None, C.byref(d), None) == -1
+    assert L.pa_copy_blocks(FAKE, FAKE, FAKE, -2, C.byref(d), None) == -1
+    assert L.pa_copy_blocks(FAKE, FAKE, FAKE, 0, C.byref(d), None) == 0
+    assert L.pa_copy_blocks(None, FAKE, FAKE, 3, C.byref(d), None) == -1
+
+
+def test_prefill_rejects_bad_arguments_on_host():
+    L = ops.lib()
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 32, 64, FAKE, FAKE, 0.1, None, None,
+                              C.byref(desc(dt=1)), None) == -2  # fp8 prefill not built
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 30, 64, FAKE, FAKE, 0.1, None, None,
+                              C.byref(desc()), None) == -1
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 32, 64, FAKE, FAKE, 0.1, None, None,
+                              C.byref(desc()), None) == 0
+
+
+def test_misaligned_pointers_are_rejected():
+    odd = C.c_void_p(0x10008)
+    L = ops.lib()
+    d = desc()
+    assert L.pa_write_kv(odd, FAKE, FAKE, 4, FAKE, FAKE, None, None, C.byref(d), None) == -1
+    assert L.pa_copy_blocks(odd, FAKE, FAKE, 3, C.byref(d), None) == -1

@@ -1,0 +1,175 @@
+"""GPU parity: slot-mapped write, block copy and paged decode (with split-K
+and its merge) against the fp64 CPU oracle, through the C ABI.
+
+Cache bytes and copies must be bit-exact; attention outputs must be within
+max-abs 1e-2 and mean-abs 1e-3 of the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (assert_attn_close, cache_to_device, dev, dev_bf16, dev_u8, host_bits, run_decode,
+                      to_float)
+from paged_kv_cache_408_b200 import inputs as I
+from paged_kv_cache_408_b200 import ops
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_decode(case, kc_host=None, vc_host=None, seq_lens=None, rows=None):
+    kc = case.k_cache if kc_host is None else kc_host
+    vc = case.v_cache if vc_host is None else vc_host
+    lens = case.seq_lens if seq_lens is None else seq_lens
+    q, bt = case.q, case.block_tables
+    if rows is not None:
+        q, bt, lens = q[rows], bt[rows], np.asarray(lens)[rows]
+    return oracle.decode(q, kc, vc, bt, lens, case.scale, case.k_scale, case.v_scale)
+
+
+# ------------------------------------------------------------------- tiny
+def test_tiny_write_is_bit_exact_and_decode_matches_before_and_after(cuda_device):
+    c = I.tiny_decode(0)
+    kc, vc = cache_to_device(c)
+    pre_lens = c.seq_lens - 1  # 5, 17, 33, 48
+    out = run_decode(c, kc, vc, seq_lens=pre_lens)
+    assert_attn_close(to_float(out), oracle_decode(c, seq_lens=pre_lens), "pre-write")
+
+    ops.write_kv(dev_bf16(c.new_k), dev_bf16(c.new_v), dev(c.slot_mapping, np.int64), kc, vc)
+    kh, vh = c.k_cache.copy(), c.v_cache.copy()
+    oracle.write_kv(c.new_k, c.new_v, c.slot_mapping, kh, vh)
+    assert np.array_equal(host_bits(kc), kh) and np.array_equal(host_bits(vc), vh)
+
+    out = run_decode(c, kc, vc)
+    assert_attn_close(to_float(out), oracle_decode(c, kh, vh), "post-write")
+    assert ops.get_last_device_error() == 0
+
+
+# ------------------------------------------------------------ shape sweep
+LENS = [1, 2, 15, 16, 17, 31, 33, 100, 255, 256, 257, 600, 1024, 1111]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_shapes(cuda_device, D, G, fp8):
+    Hkv = 2
+    c = I.make_decode_case(100 + D + 10 * G + fp8, LENS, G * Hkv, Hkv, D, fp8=fp8)
+    kc, vc = cache_to_device(c)
+    ref = oracle_decode(c)
+    for part in (0, 16, 48, 512, 2048):
+        out = run_decode(c, kc, vc, partition_tokens=part)
+        assert_attn_close(to_float(out), ref, f"D{D} G{G} fp8={fp8} P={part}")
+    assert ops.get_last_device_error() == 0
+
+
+def test_decode_zero_length_rows_are_zero(cuda_device):
+    c = I.make_decode_case(7, [0, 5, 0, 300], 8, 2, 128)
+    kc, vc = cache_to_device(c)
+    for part in (0, 16):
+        out = to_float(run_decode(c, kc, vc, partition_tokens=part))
+        assert not out[0].any() and not out[2].any()
+        assert_attn_close(out, oracle_decode(c), "zero-length rows")
+
+
+def test_decode_is_batch_invariant(cuda_device):
+    """A sequence's output does not depend on what else is in the batch."""
+    c = I.make_decode_case(8, [700, 33, 1500, 5, 260], 32, 8, 128)
+    kc, vc = cache_to_device(c)
+    full = host_bits(run_decode(c, kc, vc))
+    for rows in ([2], [4, 2, 0], [1, 3]):
+        rows = np.array(rows)
+        sub = host_bits(run_decode(c, kc, vc, seq_lens=c.seq_lens[rows], block_tables=c.block_tables[rows],
+                                   q=c.q[rows]))
+        assert np.array_equal(sub, full[rows])
+
+
+# --------------------------------------------------------- fp8 write, copy
+def test_fp8_write_is_bit_exact(cuda_device):
+    rng = np.random.default_rng(5)
+    nb, Hkv, D, T = 40, 8, 128, 300
+    ks = rng.uniform(0.002, 0.05, Hkv).astype(np.float32)
+    vs = rng.uniform(0.002, 0.05, Hkv).astype(np.float32)
+    k = I.bf16_bits(rng.standard_normal((T, Hkv, D), dtype=np.float32) * 4)
+    v = I.bf16_bits(rng.standard_normal((T, Hkv, D), dtype=np.float32) * 4)
+    k[0, 0, :4] = I.bf16_bits(np.float32([1e30, -1e30, 0.0, -0.0]))  # saturation and signed zero
+    slots = rng.permutation(nb * 16)[:T].astype(np.int64)
+    slots[::17] = -1  # padding tokens
+    kh = rng.integers(0, 255, (nb, Hkv, 16, D)).astype(np.uint8)
+    vh = rng.integers(0, 255, (nb, Hkv, 16, D)).astype(np.uint8)
+    kd, vd = dev_u8(kh), dev_u8(vh)
+    ops.write_kv(dev_bf16(k), dev_bf16(v), dev(slots, np.int64), kd, vd, dev(ks, np.float32), dev(vs, np.float32))
+    oracle.write_kv(k, v, slots, kh, vh, ks, vs)
+    assert np.array_equal(host_bits(kd), kh) and np.array_equal(host_bits(vd), vh)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_copy_blocks_is_bit_exact(cuda_device, fp8):
+    rng = np.random.default_rng(6)
+    shape = (50, 8, 16, 128)
+    if fp8:
+        kh, vh = rng.integers(0, 255, shape).astype(np.uint8), rng.integers(0, 255, shape).astype(np.uint8)
+        kd, vd = dev_u8(kh), dev_u8(vh)
+    else:
+        kh, vh = I.normal_bf16(rng, shape), I.normal_bf16(rng, shape)
+        kd, vd = dev_bf16(kh), dev_bf16(vh)
+    perm = rng.permutation(50)
+    pairs = np.stack([perm[:12], perm[12:24]], 1).astype(np.int32)
+    ops.copy_blocks(kd, vd, dev(pairs, np.int32))
+    oracle.copy_blocks(kh, vh, pairs)
+    assert np.array_equal(host_bits(kd), kh) and np.array_equal(host_bits(vd), vh)
+
+
+# ------------------------------------------------- full-size workloads
+def test_batch64_2k_full_size_sampled(cuda_device):
+    c = I.batch64_2k(0)
+    kc, vc = cache_to_device(c)
+    ops.write_kv(dev_bf16(c.new_k), dev_bf16(c.new_v), dev(c.slot_mapping, np.int64), kc, vc)
+    kh, vh = c.k_cache.copy(), c.v_cache.copy()
+    oracle.write_kv(c.new_k, c.new_v, c.slot_mapping, kh, vh)
+    assert np.array_equal(host_bits(kc), kh) and np.array_equal(host_bits(vc), vh)
+    out = to_float(run_decode(c, kc, vc))
+    rows = np.random.default_rng(1).choice(c.B, 12, replace=False)
+    rows = np.union1d(rows, [int(np.argmax(c.seq_lens)), int(np.argmin(c.seq_lens))])
+    assert_attn_close(out[rows], oracle_decode(c, kh, vh, rows=rows), "64 x U[1,2048]")
+
+
+def test_long_context_split_k_sampled(cuda_device):
+    c = I.long_context(0)
+    kc, vc = cache_to_device(c)
+    out = to_float(run_decode(c, kc, vc))
+    rows = np.array([0, 9])
+    assert_attn_close(out[rows], oracle_decode(c, rows=rows), "16 x 32768")
+    assert ops.get_last_device_error() == 0
+
+
+def test_prefix_share_fp8_sampled(cuda_device):
+    c = I.prefix_share(0)
+    kc, vc = cache_to_device(c)
+    out = to_float(run_decode(c, kc, vc))
+    rows = np.random.default_rng(2).choice(c.B, 12, replace=False)
+    assert_attn_close(out[rows], oracle_decode(c, rows=rows), "256 seqs, shared 2048 prefix, fp8")
+
+
+# ------------------------------------------------ device-side bounds checks
+def test_bad_block_id_is_flagged_not_faulted(cuda_device):
+    c = I.make_decode_case(9, [40, 40], 8, 2, 128, num_blocks=10)
+    kc, vc = cache_to_device(c)
+    assert ops.get_last_device_error() == 0
+    bt = c.block_tables.copy()
+    bt[1, 1] = 10_000  # outside the pool
+    out = to_float(run_decode(c, kc, vc, block_tables=bt))
+    assert ops.get_last_device_error() & ops.DEVERR_BAD_BLOCK
+    assert_attn_close(out[:1], oracle_decode(c, rows=np.array([0])), "unaffected row")
+
+
+def test_bad_slot_and_bad_length_are_flagged(cuda_device):
+    c = I.tiny_decode(1)
+    kc, vc = cache_to_device(c)
+    sm = c.slot_mapping.copy()
+    sm[0] = 32 * 16 + 3  # past the last block
+    ops.write_kv(dev_bf16(c.new_k), dev_bf16(c.new_v), dev(sm, np.int64), kc, vc)
+    assert ops.get_last_device_error() & ops.DEVERR_BAD_SLOT
+    lens = c.seq_lens.copy()
+    lens[2] = 10_000  # longer than the block table
+    run_decode(c, kc, vc, seq_lens=lens)
+    assert ops.get_last_device_error() & ops.DEVERR_BAD_LEN
