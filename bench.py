@@ -1,0 +1,537 @@
+"""Benchmark: paged decode KV-read GB/s and seq-steps/s on a continuous-batching trace.
+
+Default workload: 64 sequences, lengths uniform in [1, 2048], 32 q heads / 8 kv
+heads, head_dim 128, bf16 cache, sequences ending after Geometric(1/256)
+decode steps and replaced from a queue (the scheduler of
+paged_kv_cache_408_b200.runtime drives every step).  One step = copy_blocks
+(copy-on-write pairs, if any) + write_kv (the step's new K/V: one token per
+decoding sequence plus the prompts of admitted sequences) + decode (+ its
+split-K merge) [+ chunked prefill in the mixed workload].
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank runs its own independent replica of the
+trace (per-GPU work fixed: weak scaling, no collective on the data path);
+value is the work of all ranks over the slowest rank's time.  Rank 0 prints
+one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+FALLBACK_HBM_GBS = 6650.0
+
+METRIC = "paged decode KV-read GB/s (% of B200 HBM peak); seq-steps/s at 64x2K GQA"
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def file_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file, workload):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current source of the kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(workload)
+        if d and d.get("source_sha") == file_sha(os.path.join(ROOT, kernel_file)):
+            return d.get("dram_bytes_per_launch")
+    except (ValueError, OSError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = [x.strip() for x in vis.split(",")] if vis else []
+        self.gpu = ids[gpu_index] if gpu_index < len(ids) else str(gpu_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
+        loaded = [r[0] for r in rows if r[0] > 0.5 * r[1]] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+class L2Flush:
+    """Evict the L2 between timed steps: write a buffer larger than L2, then
+    read another one, so the next step starts with no useful data cached and
+    no dirty lines left to write back."""
+
+    def __init__(self, torch, device):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.sink = self.r.sum()
+
+
+def kv_bytes(lens, Hkv, D, eb):
+    return int(np.asarray(lens, np.int64).sum()) * Hkv * D * 2 * eb
+
+
+def decode_alg_bytes(lens, Hq, Hkv, D, eb):
+    lens = np.asarray(lens, np.int64)
+    B = len(lens)
+    return (kv_bytes(lens, Hkv, D, eb) + 2 * B * Hq * D * 2 + int(((lens + 15) // 16).sum()) * 4 + B * 4)
+
+
+# ----------------------------------------------------------------- workloads
+def _traces():
+    from paged_kv_cache_408_b200 import traces
+    return {"batch64_2k": traces.batch64_2k, "prefix_share_fp8": traces.prefix_share_fp8, "mixed": traces.mixed,
+            "long_context": traces.long_context}
+
+
+class _Lazy(dict):
+    def __missing__(self, k):
+        self.update(_traces())
+        return dict.__getitem__(self, k)
+
+
+TRACES = _Lazy()
+
+
+# ----------------------------------------------------------------- our arm
+class DeviceStep:
+    """One planned step's metadata as device (or pinned host) tensors."""
+
+    def __init__(self, plan, torch, device, pin=False):
+        def t(a, dt):
+            x = torch.from_numpy(np.ascontiguousarray(a, dt))
+            if pin:
+                return x.pin_memory()
+            return x.to(device)
+
+        self.plan = plan
+        self.copies = t(plan.copies, np.int32)
+        self.slots = t(plan.slots, np.int64)
+        self.tables = t(plan.decode_tables, np.int32)
+        self.lens = t(plan.decode_lens, np.int32)
+        self.p_cu = t(plan.prefill_cu, np.int32)
+        self.p_prefix = t(plan.prefill_prefix, np.int32)
+        self.p_tables = t(plan.prefill_tables, np.int32)
+        self.T = len(plan.slots)
+        self.B = plan.num_decode
+        self.nchunks = len(plan.prefill_ids)
+
+    def to(self, device, non_blocking=True):
+        d = object.__new__(DeviceStep)
+        d.__dict__.update(self.__dict__)
+        for k in ("copies", "slots", "tables", "lens", "p_cu", "p_prefix", "p_tables"):
+            setattr(d, k, getattr(self, k).to(device, non_blocking=non_blocking))
+        return d
+
+    def nbytes(self):
+        return sum(getattr(self, k).numel() * getattr(self, k).element_size()
+                   for k in ("copies", "slots", "tables", "lens", "p_cu", "p_prefix", "p_tables"))
+
+
+def run_ours(args, rank, world, device):
+    import torch
+
+    from paged_kv_cache_408_b200 import ops, traces
+
+    torch.cuda.set_device(device)
+    tr = TRACES[args.workload](args.seed + rank)
+    Hq, Hkv, D, fp8 = tr.Hq, tr.Hkv, tr.D, tr.fp8
+    eb = 1 if fp8 else 2
+    pool = tr.sched.alloc.num_blocks
+    t_plan = time.perf_counter()
+    plans = tr.plans(args.warmup + args.steps)
+    t_plan = (time.perf_counter() - t_plan) / len(plans)
+
+    g = torch.Generator(device=device).manual_seed(1234 + rank)
+    shape = (pool, Hkv, 16, D)
+    if fp8:
+        k_cache = torch.randint(0, 120, shape, dtype=torch.uint8, device=device, generator=g)
+        v_cache = torch.randint(0, 120, shape, dtype=torch.uint8, device=device, generator=g)
+        k_scale = torch.full((Hkv,), 0.01, device=device)
+        v_scale = torch.full((Hkv,), 0.01, device=device)
+    else:
+        k_cache = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+        v_cache = torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+        k_scale = v_scale = None
+    Tmax = max(p.slots.shape[0] for p in plans)
+    Bmax = max(p.num_decode for p in plans)
+    Pmax_tok = max(p.num_prefill_tokens for p in plans)
+    new_k = torch.randn((max(Tmax, 1), Hkv, D), generator=g, device=device).to(torch.bfloat16)
+    new_v = torch.randn((max(Tmax, 1), Hkv, D), generator=g, device=device).to(torch.bfloat16)
+    q = torch.randn((max(Bmax, 1), Hq, D), generator=g, device=device).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    pq = torch.randn((max(Pmax_tok, 1), Hq, D), generator=g, device=device).to(torch.bfloat16)
+    pout = torch.empty_like(pq)
+    maxb = plans[0].decode_tables.shape[1]
+    ws = ops.alloc_workspace(max(Bmax, 1), Hq, D, maxb, args.partition, device=device)
+    flush = L2Flush(torch, device)
+    scale = 1.0 / math.sqrt(D)
+    run_prefill = args.workload == "mixed"
+
+    def launch(ds, qq, oo, nk, nv, pqq, poo):
+        n = 0
+        if ds.copies.shape[0]:
+            ops.copy_blocks(k_cache, v_cache, ds.copies)
+            n += 1
+        if ds.T:
+            ops.write_kv(nk[:ds.T], nv[:ds.T], ds.slots, k_cache, v_cache, k_scale, v_scale)
+            n += 1
+        return n
+
+    def decode(ds, qq, oo):
+        if ds.B:
+            ops.decode(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.tables, ds.lens, scale, k_scale, v_scale, ws,
+                       args.partition)
+            return 2  # decode kernel + merge kernel
+        return 0
+
+    def prefill(ds, pqq, poo):
+        if run_prefill and ds.nchunks:
+            nt = int(ds.plan.prefill_cu[-1])
+            ops.prefill_chunk(poo[:nt], pqq[:nt], ds.p_cu, ds.p_prefix, ds.p_tables, k_cache, v_cache, scale,
+                              ds.plan.max_chunk)
+            return 1
+        return 0
+
+    dsteps = [DeviceStep(p, torch, device) for p in plans]
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+
+    # ---- warm-up
+    for ds in dsteps[:args.warmup]:
+        launch(ds, q, out, new_k, new_v, pq, pout)
+        decode(ds, q, out)
+        prefill(ds, pq, pout)
+    torch.cuda.synchronize()
+    if ops.get_last_device_error() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    # ---- timed: inputs resident in HBM, L2 flushed between steps (outside the events)
+    timed = dsteps[args.warmup:]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
+    launches = 0
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        # hold the stream while the host enqueues every timed step, so the
+        # events see device time only (no host launch gaps)
+        torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
+        for ds, (e0, e1, e2, e3) in zip(timed, ev):
+            flush()
+            e0.record(st)
+            launches += launch(ds, q, out, new_k, new_v, pq, pout)
+            e1.record(st)
+            launches += decode(ds, q, out)
+            e2.record(st)
+            launches += prefill(ds, pq, pout)
+            e3.record(st)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [e0.elapsed_time(e3) for e0, _, _, e3 in ev]
+    dec_ms = [e1.elapsed_time(e2) for _, e1, e2, _ in ev]
+    tot_ms = sum(step_ms)
+    kvb = sum(kv_bytes(ds.plan.decode_lens, Hkv, D, eb) for ds in timed)
+    seqsteps = sum(ds.B for ds in timed)
+    algb = [decode_alg_bytes(ds.plan.decode_lens, Hq, Hkv, D, eb) for ds in timed if ds.B]
+    flags = ops.get_last_device_error()
+    if flags:
+        raise RuntimeError(f"device status word {flags:#x} after the timed steps")
+
+    # ---- end to end: per-step inputs from pinned host memory, result read back
+    e2e = None
+    if not args.no_e2e:
+        hsteps = [DeviceStep(p, torch, device, pin=True) for p in plans[args.warmup:]]
+        hq = q.cpu().pin_memory()
+        hk = new_k.cpu().pin_memory()
+        hv = new_v.cpu().pin_memory()
+        hout = torch.empty_like(hq).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(new_k), torch.empty_like(new_v)
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in hsteps]
+        h2d = d2h = 0
+        torch.cuda.synchronize()
+        for hs, (e0, e1) in zip(hsteps, ee):
+            flush()
+            e0.record(st)
+            ds = hs.to(device)
+            nq, nt = hs.B * Hq * D * 2, hs.T * Hkv * D * 2
+            if hs.B:
+                dq[:hs.B].copy_(hq[:hs.B], non_blocking=True)
+            if hs.T:
+                dk[:hs.T].copy_(hk[:hs.T], non_blocking=True)
+                dv[:hs.T].copy_(hv[:hs.T], non_blocking=True)
+            launch(ds, dq, out, dk, dv, pq, pout)
+            decode(ds, dq, out)
+            prefill(ds, pq, pout)
+            if hs.B:
+                hout[:hs.B].copy_(out[:hs.B], non_blocking=True)
+            e1.record(st)
+            h2d += hs.nbytes() + nq + 2 * nt
+            d2h += hs.B * Hq * D * 2
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
+        e2e = {"ms": e2e_ms, "h2d": h2d / len(hsteps), "d2h": d2h / len(hsteps), "kvb": kvb}
+
+    return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb,
+                launches=launches, clocks=clk.summary(), e2e=e2e, plan_ms=t_plan * 1e3, tr=tr, plans=plans,
+                k_cache=k_cache, v_cache=v_cache, Hq=Hq, Hkv=Hkv, D=D, eb=eb, fp8=fp8, scale=scale,
+                k_scale=k_scale, v_scale=v_scale, q=q, pool=pool)
+
+
+# ------------------------------------------------------------ oracle timing
+def oracle_step_time(plan, kc, vc, q, Hq, scale, ks, vs, rows, nthreads):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.decode(q[rows], kc, vc, plan.decode_tables[rows], plan.decode_lens[rows], scale, ks, vs,
+                  nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_from(plans, kc, vc, qh, Hq, Hkv, D, eb, scale, ks, vs, budget_s=15.0):
+    """Time the fp64 oracle, as it stands, on whole steps of the same trace
+    until about ``budget_s`` seconds of CPU work are done."""
+    import oracle
+    nthreads = os.cpu_count() or 1
+    done_b = 0
+    secs = 0.0
+    nsteps = 0
+    for p in plans:
+        rows = np.arange(p.num_decode)
+        secs += oracle_step_time(p, kc, vc, qh[:p.num_decode], Hq, scale, ks, vs, rows, nthreads)
+        done_b += kv_bytes(p.decode_lens, Hkv, D, eb)
+        nsteps += 1
+        if secs >= budget_s:
+            break
+    used = oracle.max_threads()
+    return {"value": done_b / secs / 1e9, "unit": "GB/s", "cores": used, "kind": "oracle",
+            "sample": f"{nsteps} whole decode steps of the same trace (fp64 C oracle, OpenMP over sequence x "
+                      f"head), {secs:.1f} s", "seq_steps_per_s": sum(p.num_decode for p in plans[:nsteps]) / secs}
+
+
+def host_copy(t, torch):
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    """The oracle timed as the reference arm on the host cores."""
+    if rank != 0:
+        return None
+    from paged_kv_cache_408_b200 import traces, inputs as I
+    import oracle
+    tr = TRACES[args.workload](args.seed)
+    plans = tr.plans(args.warmup + args.steps)
+    rng = np.random.default_rng(7)
+    shape = (tr.sched.alloc.num_blocks, tr.Hkv, 16, tr.D)
+    if tr.fp8:
+        kc = rng.integers(0, 120, shape).astype(np.uint8)
+        vc = rng.integers(0, 120, shape).astype(np.uint8)
+        ks = np.full(tr.Hkv, 0.01, np.float32)
+        vs = ks.copy()
+    else:
+        kc, vc = I.normal_bf16(rng, shape), I.normal_bf16(rng, shape)
+        ks = vs = None
+    eb = 1 if tr.fp8 else 2
+    Bmax = max(p.num_decode for p in plans)
+    qh = I.normal_bf16(rng, (Bmax, tr.Hq, tr.D))
+    scale = 1.0 / math.sqrt(tr.D)
+    nthreads = os.cpu_count() or 1
+    # bounded sample per step: the first `rows` sequences of each step, sized
+    # so one step takes about 2 s on these cores
+    probe = plans[0]
+    t1 = oracle_step_time(probe, kc, vc, qh, tr.Hq, scale, ks, vs, np.arange(min(8, probe.num_decode)), nthreads)
+    per_seq = t1 / min(8, probe.num_decode)
+    nrows = int(max(1, min(Bmax, 2.0 / max(per_seq, 1e-6))))
+    for p in plans[:args.warmup]:
+        oracle_step_time(p, kc, vc, qh, tr.Hq, scale, ks, vs, np.arange(min(nrows, p.num_decode)), nthreads)
+    secs = 0.0
+    kvb = 0
+    seqsteps = 0
+    for p in plans[args.warmup:]:
+        rows = np.arange(min(nrows, p.num_decode))
+        secs += oracle_step_time(p, kc, vc, qh, tr.Hq, scale, ks, vs, rows, nthreads)
+        kvb += kv_bytes(p.decode_lens[rows], tr.Hkv, tr.D, eb)
+        seqsteps += len(rows)
+    value = kvb / secs / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args, tr),
+            "seq_steps_per_s": seqsteps / secs,
+            "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": oracle.max_threads(),
+                             "sample": f"first {nrows} sequences of each step of the same trace"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+def workload_config(args, tr):
+    return {"workload": tr.name, "trace": args.workload, "seqs": tr.sched.cfg.max_num_seqs, "q_heads": tr.Hq,
+            "kv_heads": tr.Hkv, "head_dim": tr.D, "block_size": 16, "cache_dtype": "fp8_e4m3" if tr.fp8 else "bf16",
+            "pool_blocks": tr.sched.alloc.num_blocks, "partition_tokens": args.partition or 256,
+            "l2": "flushed between steps outside the timed events (256 MiB written, then 256 MiB read)", "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------- driver
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["batch64_2k", "prefix_share_fp8", "mixed", "long_context"],
+                    default="batch64_2k")
+    ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    device = torch.device(f"cuda:{local}")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(device)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    r = run_ours(args, rank, world, device)
+
+    tot_s = r["tot_ms"] / 1e3
+    kvb, seqsteps = r["kvb"], r["seqsteps"]
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([tot_s], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        w = torch.tensor([kvb, seqsteps], device=device, dtype=torch.float64)
+        dist.all_reduce(w, op=dist.ReduceOp.SUM)
+        tot_s = float(t.item())
+        kvb, seqsteps = float(w[0].item()), float(w[1].item())
+
+    if rank == 0:
+        peak, peak_kind = peaks()
+        dec_ms = sum(r["dec_ms"]) / len(r["dec_ms"])
+        alg = sum(r["algb"]) / len(r["algb"])
+        achieved = alg / (dec_ms / 1e3) / 1e9
+        tr = r["tr"]
+        line = {
+            "metric": METRIC, "value": kvb / tot_s / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["tot_ms"] / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not r["fp8"] else "fp8_e4m3",
+            "data": "synthetic", "config": workload_config(args, tr),
+            "seq_steps_per_s": seqsteps / tot_s,
+            "pct_of_hbm_peak": 100.0 * (kvb / tot_s / 1e9) / peak,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": f"{peak_kind} (copy bandwidth)", "kernel": "pa_decode (decode + merge)",
+                         "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", args.workload),
+                         "alg_bytes_per_launch": alg, "ms_per_launch": dec_ms},
+            "gpu_launches": r["launches"],
+            "clocks": r["clocks"],
+            "host_plan_ms_per_step": r["plan_ms"],
+            "preemptions": tr.sched.num_preemptions,
+        }
+        if r["e2e"] is not None:
+            e = r["e2e"]
+            line["e2e"] = {"value": e["kvb"] / (e["ms"] / 1e3) / 1e9, "unit": "GB/s",
+                           "h2d_bytes_per_step": int(e["h2d"]), "d2h_bytes_per_step": int(e["d2h"]),
+                           "ms_per_step": e["ms"] / args.steps}
+        if world == 1 and not args.no_cpu_baseline:
+            import torch as _t
+            kc, vc = host_copy(r["k_cache"], _t), host_copy(r["v_cache"], _t)
+            qh = host_copy(r["q"], _t)
+            ks = r["k_scale"].cpu().numpy() if r["k_scale"] is not None else None
+            vs = r["v_scale"].cpu().numpy() if r["v_scale"] is not None else None
+            line["cpu_baseline"] = cpu_baseline_from(r["plans"][args.warmup:], kc, vc, qh, r["Hq"], r["Hkv"],
+                                                     r["D"], r["eb"], r["scale"], ks, vs)
+        print(json.dumps(line), flush=True)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

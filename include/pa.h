@@ -139,7 +139,8 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, i
 /*
  * pa_decode_workspace_size -- bytes of device workspace pa_decode needs for
  * this shape (host function, no device work).  partition_tokens as for
- * pa_decode.
+ * pa_decode.  0 means no workspace is needed (every sequence fits one
+ * partition).
  */
 int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
                              int32_t partition_tokens, size_t *bytes);
@@ -159,17 +160,29 @@ int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head
  *   seq_lens      int32 [num_seqs]; 0 gives an all-zero output row.
  *   scale         softmax scale (typically 1/sqrt(head_dim)).
  *   k_scale, v_scale  fp32 [num_kv_heads] for an fp8 cache, else ignored.
- *   partition_tokens  split-K partition length in tokens: a multiple of 16
- *                 in [16, 4096], or 0 for the library default (256).  Each
- *                 partition of a sequence yields a partial result and its
- *                 log-sum-exp; sequences with more than one partition are
- *                 combined by a log-sum-exp merge.  Partition boundaries
- *                 depend only on the token index, so a sequence's result
- *                 does not depend on the rest of the batch.
+ *   partition_tokens  how a sequence's tokens are split across CTAs
+ *                 (split-K; the pieces are combined by a log-sum-exp merge
+ *                 inside the same kernel):
+ *                 0  -- balanced: the (sequence, kv head, block) work of the
+ *                       whole batch is cut into equal contiguous shares, one
+ *                       per resident CTA, so every SM streams the same
+ *                       number of bytes whatever the length mix (fastest;
+ *                       split points depend on the batch, so the last bits
+ *                       of a result can differ between batch compositions);
+ *                 16..2048, a multiple of 16 -- fixed partitions of that
+ *                       many tokens: split points depend only on token
+ *                       positions, so each sequence's result is bitwise
+ *                       independent of the rest of the batch.
  *   workspace     device scratch of at least pa_decode_workspace_size()
- *                 bytes, 256-byte aligned; contents need no initialisation
- *                 and are garbage afterwards.
- * num_seqs must be in [1, 2048]; num_q_heads / num_kv_heads in {1,2,4,8}.
+ *                 bytes, 256-byte aligned.  It must be zero-filled before
+ *                 its first use (e.g. cudaMemset); its first bytes hold the
+ *                 per-(sequence, kv head) arrival counters of the in-kernel
+ *                 split-K merge, which every completed call leaves at zero,
+ *                 so later calls (any batch size) need no re-initialisation.
+ *                 Calls that share one workspace must not overlap on the
+ *                 GPU.
+ * num_seqs must be in [0, 2048] (0 enqueues nothing); num_kv_heads <= 128;
+ * num_q_heads / num_kv_heads in {1,2,4,8}.
  */
 int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
               const int32_t *seq_lens, int32_t num_seqs, int32_t max_blocks_per_seq, int32_t num_q_heads,

@@ -14,8 +14,7 @@ __device__ unsigned pa_device_status_word;
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kDefaultPartition = 256;
-constexpr int kMaxSeqs = 2048;
+constexpr int kMaxSeqs = pa::kMaxDecodeSeqs;
 
 unsigned *status_word_ptr() {
     static std::mutex mu;
@@ -49,9 +48,10 @@ int from_cuda(cudaError_t e) {
     return PA_ERR_CUDA;
 }
 
+// 0 selects the balanced split; otherwise fixed partitions of 16..2048 tokens.
 int resolve_partition(int32_t partition_tokens, int *out) {
-    const int p = partition_tokens == 0 ? kDefaultPartition : partition_tokens;
-    if (p < 16 || p > 2048 || p % 16 != 0) return PA_ERR_INVALID_ARG;
+    const int p = partition_tokens;
+    if (p != 0 && (p < 16 || p > 2048 || p % 16 != 0)) return PA_ERR_INVALID_ARG;
     *out = p;
     return PA_OK;
 }
@@ -111,7 +111,7 @@ int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head
     int P = 0;
     int rc = resolve_partition(partition_tokens, &P);
     if (rc != PA_OK) return rc;
-    const int max_parts = (max_blocks_per_seq * 16 + P - 1) / P;
+    const int max_parts = pa::decode_max_parts(max_blocks_per_seq, P);
     *bytes = max_parts > 1 ? pa::decode_ws_bytes(num_seqs, num_q_heads, head_dim, max_parts) : 0;
     return PA_OK;
 }
@@ -125,6 +125,7 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     if (num_seqs < 0 || num_seqs > kMaxSeqs || max_blocks_per_seq <= 0 || num_q_heads <= 0)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (desc->num_kv_heads > pa::kMaxDecodeKvHeads) return PA_ERR_UNSUPPORTED;
     const int G = num_q_heads / desc->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PA_OK;
@@ -135,19 +136,22 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     int P = 0;
     rc = resolve_partition(partition_tokens, &P);
     if (rc != PA_OK) return rc;
-    const int max_parts = (max_blocks_per_seq * 16 + P - 1) / P;
+    const int max_parts = pa::decode_max_parts(max_blocks_per_seq, P);
+    int *counters = nullptr;
     float *ws_o = nullptr, *ws_lse = nullptr;
     if (max_parts > 1) {
         const size_t need = pa::decode_ws_bytes(num_seqs, num_q_heads, desc->head_dim, max_parts);
         if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
             return PA_ERR_WORKSPACE;
-        ws_o = static_cast<float *>(workspace);
-        ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+        char *base = static_cast<char *>(workspace);
+        counters = reinterpret_cast<int *>(base);
+        ws_o = reinterpret_cast<float *>(base + pa::decode_ws_counter_bytes());
+        ws_lse = reinterpret_cast<float *>(base + pa::decode_ws_counter_bytes() +
                                            pa::decode_ws_o_bytes(num_seqs, num_q_heads, desc->head_dim, max_parts));
     }
     pa::DecodeArgs a{out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
                      num_q_heads, desc->num_kv_heads, desc->head_dim, desc->num_blocks, scale, k_scale, v_scale,
-                     P, max_parts, ws_o, ws_lse, fp8, status_word_ptr()};
+                     P, max_parts, counters, ws_o, ws_lse, fp8, status_word_ptr()};
     return from_cuda(pa::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 

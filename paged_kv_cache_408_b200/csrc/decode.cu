@@ -1,5 +1,5 @@
-// decode.cu -- paged decode attention for sm_100a, with split-K partials and
-// a log-sum-exp merge.
+// decode.cu -- paged decode attention for sm_100a, with split-K pieces and
+// an in-kernel log-sum-exp merge.
 //
 // What is computed ("Production Serving: Continuous Batching and
 // PagedAttention", The Build, Step 6 "Implement attention over paged
@@ -9,34 +9,42 @@
 // block_tables[b][t/16], kv head floor(h*Hkv/Hq).
 //
 // How (B200 design):
-//  * Work unit ("item") = (sequence, kv head, partition of `P` tokens).  One
-//    CTA processes a whole GQA group for its item, so each K/V byte is read
-//    from HBM exactly once per step.  Partitions depend only on token index:
-//    a sequence's result never depends on the rest of the batch.
-//  * Persistent grid: every CTA rebuilds the item list from seq_lens in
-//    shared memory (a block-wide scan) and walks items
-//    blockIdx.x, blockIdx.x + gridDim.x, ...; full partitions come first, the
-//    ragged tails last.  No empty CTAs for short sequences, no host sync.
-//  * Each warp streams its own 16-token blocks (blocks w, w+4, ... of the
-//    item) through an NSTAGE-deep shared-memory ring filled by 1-D bulk
-//    async copies (the TMA engine, 4 KB contiguous per K or V block) that
-//    complete on mbarriers.  The producer runs ahead across item boundaries
-//    and prefetches the next item's block-table entries into registers.
-//  * Math on CUDA cores (the contraction per step is 4-8 query rows, far
-//    below a tensor-core tile): lanes are split into token groups of LPT
-//    lanes; a lane owns DPL head dims (16-byte shared-memory reads, bank-
-//    conflict-free), holds q for those dims in fp32 registers pre-scaled by
-//    scale*log2(e), and accumulates with packed fp32x2 FMAs.  Partial dot
-//    products are combined by a shuffle reduce-scatter, exponentiated by the
-//    owning lane, and all-gathered for the P.V step.
-//  * Online softmax with a lazily updated running max: the max only moves
-//    when a new score exceeds it by more than 2^8 (ratio), so the common
-//    block needs no max shuffles; final normalisation divides by the sum
-//    taken against the same max, so the result is the exact softmax.
-//  * Each token group keeps its own (m, l, acc); groups, then warps, are
-//    combined once per item.  A sequence with one partition writes bf16
-//    output directly; longer ones write fp32 partials and log2-sum-exp to
-//    the workspace, merged by merge_kernel.
+//  * The unit of work is a warp.  Every warp streams 16-token blocks of ONE
+//    (sequence, kv head) at a time and computes the whole GQA group of that
+//    kv head, so each K/V byte is read from HBM exactly once per step.
+//    Warps are independent: no CTA barrier inside the main loop, so one
+//    warp's per-item latencies (q load, epilogue, merge) are hidden by the
+//    other warps of the SM.
+//  * Work split (host selects with partition_tokens):
+//      balanced -- the (sequence, kv head, block) triples of the batch form
+//        one line; warp g takes the contiguous share [g*S, (g+1)*S) with
+//        S = ceil(total / warps): every warp streams the same number of
+//        bytes whatever the length mix;
+//      fixed -- every (sequence, kv head) is cut into partitions of P tokens,
+//        dealt round-robin to warps (full partitions first); split points
+//        depend only on token positions, so results are batch-invariant.
+//    Every CTA rebuilds the split from seq_lens with a block-wide scan in
+//    shared memory: no host sync, no empty CTAs for short sequences.
+//  * Each warp runs its own NSTAGE-deep shared-memory ring filled by 1-D
+//    bulk async copies (the TMA engine; K and V of one block of one kv head
+//    are 4 KB contiguous each) that complete on mbarriers.  The producer
+//    runs ahead across item boundaries and keeps block-table entries in
+//    registers (a sliding window, plus the next item's first entries).
+//  * Math on CUDA cores (4-8 query rows per step are far below a
+//    tensor-core tile): lanes form token groups of LPT lanes; a lane owns
+//    DPL head dims (16-byte shared-memory reads, bank-conflict-free), keeps
+//    q for them in fp32 registers pre-scaled by scale*log2(e), and
+//    accumulates with packed fp32x2 FMAs.  Partial dot products are
+//    completed by a select-free shuffle reduce-scatter, exponentiated by the
+//    owning lane and all-gathered for P.V.
+//  * Online softmax with a lazily moved running max (it only moves when a
+//    score exceeds it by more than 8 in log2 units); the final division uses
+//    the sum taken against the same max, so the result is the exact softmax.
+//  * A (sequence, kv head) covered by one piece is written as bf16 straight
+//    from registers.  Otherwise each piece writes its fp32 output and its
+//    log2-sum-exp to the workspace and bumps an arrival counter; the warp
+//    that completes the last piece merges all pieces by log-sum-exp and
+//    resets the counter (the workspace stays ready for the next call).
 #include <algorithm>
 #include <mutex>
 
@@ -61,11 +69,11 @@ struct Cfg {
     static constexpr int D = D_, G = G_;
     static constexpr bool FP8 = FP8_;
     static constexpr int EB = FP8 ? 1 : 2;           // bytes per element
-    static constexpr int DPL = (G >= 8) ? 8 : 16;     // head dims owned by a lane
+    static constexpr int DPL = (G >= 4) ? 8 : 16;     // head dims owned by a lane
     static constexpr int LPT = D / DPL;               // lanes per token
     static constexpr int NGRP = 32 / LPT;             // token groups per warp
     static constexpr int TPG = 16 / NGRP;             // tokens per group per block
-    static constexpr int TSUB = (TPG * G > 32) ? 32 / G : TPG;  // tokens per group per sub-step
+    static constexpr int TSUB = (TPG * G > 16) ? (16 / G > 0 ? 16 / G : 1) : TPG;  // tokens per sub-step
     static constexpr int NSUB = TPG / TSUB;
     static constexpr int NCH = DPL / 8;               // 8-element chunks per lane per row
     static constexpr int CHB = 8 * EB;                // bytes per chunk
@@ -77,11 +85,12 @@ struct Cfg {
     static constexpr int VPL = RS ? NS / LPT : NS;    // scores a lane owns after the reduction
     static constexpr int NW = 4;                      // warps per CTA
     static constexpr int NT = NW * 32;
-    static constexpr int NSTAGE = 3;                  // ring depth per warp
+    static constexpr int NSTAGE = (G >= 8) ? 3 : 2;   // ring depth per warp
+    static constexpr int MIN_CTAS = (G >= 8) ? 2 : 3; // resident CTAs per SM the register budget targets
     static constexpr size_t STAGE_BYTES = (size_t)NW * NSTAGE * 2 * BLKB;
-    static constexpr size_t RED_FLOATS = (size_t)NW * G * (D + 2);
     static_assert(LPT >= 1 && LPT <= 32 && 32 % LPT == 0, "bad lane split");
     static_assert(TPG * NGRP == 16 && TSUB * NSUB == TPG, "bad token split");
+    static_assert(!RS || NS % LPT == 0, "reduce-scatter needs NS divisible by LPT");
 };
 
 template <class C>
@@ -89,9 +98,8 @@ size_t smem_bytes(int B) {
     size_t s = C::STAGE_BYTES;
     s += (size_t)C::NW * C::NSTAGE * 8;   // mbarriers
     s += (size_t)C::NW * C::NSTAGE * 4;   // valid-token count per stage
-    s = (s + 15) & ~(size_t)15;
-    s += C::RED_FLOATS * 4;               // cross-warp combine
-    s += (size_t)(3 * B + 2) * 4;         // lens, full-partition scan, tail scan
+    s += (size_t)2 * C::NW * 4;           // scan scratch
+    s += (size_t)(3 * B + 2) * 4;         // lens and two exclusive scans
     return s;
 }
 
@@ -105,31 +113,385 @@ PA_DEVICE int upper_index(const int *arr, int n, int u) {
     return lo;
 }
 
+// ---- compile-time butterflies over the LPT lanes of a token group.
+//
+// Lane `sub` of a group stores partial score idx (= token*G + head within a
+// sub-step) at register position idx ^ S, S = sub*VPL.  With that lane-
+// dependent layout a reduce-scatter is select-free: at every level a lane
+// keeps positions [0, N) and adds the partner's positions [N, 2N), and after
+// the last level positions [0, VPL) hold the lane's own complete scores
+// (idx = S + i).  The all-gather walks back the same way.  The layout costs
+// nothing: the XOR on the head bits permutes which q head sits in which
+// register slot (chosen once, at the q load), the XOR on the token bits
+// permutes which shared-memory row a lane reads.
+template <int MASK, int N, int NS>
+PA_DEVICE void rs_level(float (&v)[NS]) {
+    if constexpr (MASK >= 1) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) v[k] += __shfl_xor_sync(kFull, v[k + N], MASK);
+        rs_level<MASK / 2, N / 2, NS>(v);
+    }
+}
+
+template <int MASK, int LPT, int N, int NS>
+PA_DEVICE void ag_level(float (&v)[NS]) {
+    if constexpr (MASK < LPT) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) v[k + N] = __shfl_xor_sync(kFull, v[k], MASK);
+        ag_level<MASK * 2, LPT, N * 2, NS>(v);
+    }
+}
+
+// Butterfly all-reduce (sum) of NS values over lanes whose index differs in
+// bits below LPT (used when every lane keeps every score).
+template <int MASK, int NS>
+PA_DEVICE void allreduce_level(float (&v)[NS]) {
+    if constexpr (MASK >= 1) {
+#pragma unroll
+        for (int k = 0; k < NS; ++k) v[k] += __shfl_xor_sync(kFull, v[k], MASK);
+        allreduce_level<MASK / 2, NS>(v);
+    }
+}
+
+// All-reduce of per-head values kept in permuted head slots: slot h of lane
+// sub is head h ^ (sub*VPL % G), so the partner across MASK keeps my head in
+// slot h ^ (MASK*VPL % G).  MAX selects max, otherwise sum.
+template <int MASK, int VPL, int G, bool MAX>
+PA_DEVICE void perm_allreduce(float (&v)[G]) {
+    if constexpr (MASK >= 1) {
+        constexpr int X = (MASK * VPL) % G;
+        float r[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) r[h] = __shfl_xor_sync(kFull, v[h ^ X], MASK);
+#pragma unroll
+        for (int h = 0; h < G; ++h) v[h] = MAX ? fmaxf(v[h], r[h]) : v[h] + r[h];
+        perm_allreduce<MASK / 2, VPL, G, MAX>(v);
+    }
+}
+
+// Merge the (m, l, acc) states of token groups: partners differ in the group
+// bits (MASK = LPT, 2*LPT, ... 16).  Groups of opposite parity visit their
+// two 16-byte chunks in swapped order, so at MASK == LPT the partner's
+// register holding my chunk is at the other half (k ^ 4).
+template <int MASK, int LPT, int G, int P2, bool SWAP>
+PA_DEVICE void group_merge(float (&m)[G], float (&l)[G], float2 (&acc)[G][P2]) {
+    if constexpr (MASK < 32) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float mo = __shfl_xor_sync(kFull, m[h], MASK);
+            const float lo = __shfl_xor_sync(kFull, l[h], MASK);
+            const float M = fmaxf(m[h], mo);
+            const float am = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - M);
+            const float ao = (mo == -INFINITY) ? 0.f : ex2(mo - M);
+            l[h] = l[h] * am + lo * ao;
+            m[h] = M;
+            float2 rx[P2];
+#pragma unroll
+            for (int k = 0; k < P2; ++k) {
+                constexpr bool sw = SWAP && MASK == LPT;
+                const int ks = sw ? (k ^ 4) : k;
+                rx[k].x = __shfl_xor_sync(kFull, acc[h][ks].x, MASK);
+                rx[k].y = __shfl_xor_sync(kFull, acc[h][ks].y, MASK);
+            }
+#pragma unroll
+            for (int k = 0; k < P2; ++k)
+                acc[h][k] = ffma2(acc[h][k], make_float2(am, am), make_float2(rx[k].x * ao, rx[k].y * ao));
+        }
+        group_merge<MASK * 2, LPT, G, P2, SWAP>(m, l, acc);
+    }
+}
+
+// A unit of work: blocks [blk0, blk0 + nblk) of sequence b, kv head kvh.
+// It is piece `piece` of the npieces pieces that cover that (sequence, kv
+// head); a single piece writes the output, several pieces are merged.
 struct Item {
-    int b, kvh, part, len, blk0, nblk, nparts;
+    int b, kvh, piece, npieces, len, blk0, nblk;
+};
+
+// The work split, rebuilt by every CTA from seq_lens in shared memory.
+struct Schedule {
+    const int *len;   // [B]
+    const int *pre0;  // balanced: segment offset [B+1]; fixed: full-partition prefix [B+1]
+    const int *pre1;  // fixed: tail prefix [B+1]
+    int B, Hkv, P;
+    int total;        // balanced: blocks in the line; fixed: number of items
+    int S;            // balanced: share per warp, in blocks
+    int NF;           // fixed: number of full-partition entries (per kv head)
+
+    PA_DEVICE Item fixed_item(int i) const {
+        Item it;
+        it.kvh = i % Hkv;
+        int u = i / Hkv;
+        if (u < NF) {
+            it.b = upper_index(pre0, B, u);
+            it.piece = u - pre0[it.b];
+        } else {
+            u -= NF;
+            it.b = upper_index(pre1, B, u);
+            it.piece = pre0[it.b + 1] - pre0[it.b];
+        }
+        it.len = len[it.b];
+        it.npieces = (pre0[it.b + 1] - pre0[it.b]) + (pre1[it.b + 1] - pre1[it.b]);
+        const int t0 = it.piece * P, t1 = min(t0 + P, it.len);
+        it.blk0 = t0 >> 4;
+        it.nblk = ((t1 + 15) >> 4) - it.blk0;
+        return it;
+    }
+
+    // balanced: the piece that starts at line position pos, cut at `end`
+    PA_DEVICE Item balanced_item(int pos, int end) const {
+        Item it;
+        it.b = upper_index(pre0, B, pos);
+        it.len = len[it.b];
+        const int nb = (it.len + 15) >> 4;
+        const int u = pos - pre0[it.b];
+        it.kvh = u / nb;
+        it.blk0 = u - it.kvh * nb;
+        const int seg0 = pre0[it.b] + it.kvh * nb, seg1 = seg0 + nb;
+        it.nblk = min(seg1, end) - pos;
+        it.piece = pos / S - seg0 / S;
+        it.npieces = (seg1 - 1) / S - seg0 / S + 1;
+        return it;
+    }
+};
+
+// Walks the items of one warp (global warp index gw of GW) in order.
+struct ItemIter {
+    int cur, end, step;
+
+    PA_DEVICE void start(const Schedule &sc, int gw, int GW) {
+        if (sc.P == 0) {
+            cur = min(sc.total, gw * sc.S);
+            end = min(sc.total, cur + sc.S);
+            step = 0;
+        } else {
+            cur = gw;
+            end = sc.total;
+            step = GW;
+        }
+    }
+    PA_DEVICE bool next(const Schedule &sc, Item &it) {
+        if (cur >= end) return false;
+        if (sc.P == 0) {
+            it = sc.balanced_item(cur, end);
+            cur += it.nblk;
+        } else {
+            it = sc.fixed_item(cur);
+            cur += step;
+        }
+        return true;
+    }
+};
+
+// Per-warp producer: lane 0 issues the two bulk copies (K and V block of one
+// kv head) for the next block of the warp's stream.  The warp keeps a
+// 64-entry window of the current item's block-table entries in registers
+// (lane l holds entries base+l and base+32+l), slid 32 entries ahead of use,
+// plus the first 64 entries of the next item, loaded while the current one
+// streams.
+template <class C>
+struct Producer {
+    ItemIter iter;
+    Item cur, nxt;
+    bool has_cur, has_nxt;
+    int j, base;
+    int t0, t1, nt0, nt1;
+    uint32_t issued;
+
+    PA_DEVICE int load32(const DecodeArgs &a, const Item &it, int lane, int off) {
+        const int32_t *row = a.block_tables + (size_t)it.b * a.max_blocks + it.blk0;
+        return (off + lane < it.nblk) ? row[off + lane] : -1;
+    }
+
+    PA_DEVICE void fetch_next(const Schedule &sc, const DecodeArgs &a, int lane) {
+        has_nxt = iter.next(sc, nxt);
+        if (has_nxt) {
+            nt0 = load32(a, nxt, lane, 0);
+            nt1 = load32(a, nxt, lane, 32);
+        }
+    }
+
+    PA_DEVICE void advance(const Schedule &sc, const DecodeArgs &a, int lane) {
+        cur = nxt;
+        has_cur = has_nxt;
+        t0 = nt0;
+        t1 = nt1;
+        j = 0;
+        base = 0;
+        fetch_next(sc, a, lane);
+    }
+
+    PA_DEVICE void init(const Schedule &sc, const DecodeArgs &a, int gw, int GW, int lane) {
+        issued = 0;
+        iter.start(sc, gw, GW);
+        fetch_next(sc, a, lane);
+        advance(sc, a, lane);
+    }
+
+    PA_DEVICE void produce(const Schedule &sc, const DecodeArgs &a, int lane, const uint8_t *kc, const uint8_t *vc,
+                           uint8_t *stg, uint64_t *bars, int *valid_of) {
+        while (has_cur && j >= cur.nblk) advance(sc, a, lane);
+        if (!has_cur) return;
+        if (j - base == 32) {  // slide the window: refill 32 entries ahead
+            t0 = t1;
+            t1 = load32(a, cur, lane, base + 64);
+            base += 32;
+        }
+        int phys = __shfl_sync(kFull, t0, j - base);
+        if (lane == 0) {
+            const int blk = cur.blk0 + j;
+            int valid = min(16, cur.len - blk * 16);
+            if (phys < 0 || phys >= a.num_blocks) {
+                flag_error(a.err, PA_DEVERR_BAD_BLOCK);
+                phys = 0;
+                valid = 0;
+            }
+            const int s = issued % C::NSTAGE;
+            valid_of[s] = valid;
+            mbar_arrive_expect_tx(&bars[s], 2 * C::BLKB);
+            const size_t src = ((size_t)phys * sc.Hkv + cur.kvh) * C::BLKB;
+            uint8_t *dst = stg + (size_t)s * 2 * C::BLKB;
+            bulk_g2s(dst, kc + src, C::BLKB, &bars[s]);
+            bulk_g2s(dst + C::BLKB, vc + src, C::BLKB, &bars[s]);
+        }
+        ++issued;
+        ++j;
+    }
+};
+
+// Load this lane's chunks of one token row from shared memory and widen to fp32 pairs.
+template <class C>
+PA_DEVICE void load_row(const uint8_t *row, const int (&choff)[C::NCH], float2 (&f)[C::P2]) {
+#pragma unroll
+    for (int c = 0; c < C::NCH; ++c) {
+        if constexpr (!C::FP8) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(row + choff[c] * C::CHB);
+            f[4 * c + 0] = bf16x2_to_float2(u.x);
+            f[4 * c + 1] = bf16x2_to_float2(u.y);
+            f[4 * c + 2] = bf16x2_to_float2(u.z);
+            f[4 * c + 3] = bf16x2_to_float2(u.w);
+        } else {
+            const uint2 u = *reinterpret_cast<const uint2 *>(row + choff[c] * C::CHB);
+            f[4 * c + 0] = e4m3x2_to_float2((uint16_t)(u.x & 0xffff));
+            f[4 * c + 1] = e4m3x2_to_float2((uint16_t)(u.x >> 16));
+            f[4 * c + 2] = e4m3x2_to_float2((uint16_t)(u.y & 0xffff));
+            f[4 * c + 3] = e4m3x2_to_float2((uint16_t)(u.y >> 16));
+        }
+    }
+}
+
+// Log-sum-exp merge of the npieces partial results of one (sequence, kv
+// head) by a single warp: out = sum_p w_p o_p / sum_p w_p with
+// w_p = 2^(lse_p - max lse).  Pieces are read in chunks of CH with every load
+// of a chunk in flight at once (one L2 round trip per chunk, all heads
+// together); the running max is moved between chunks.
+template <class C>
+PA_DEVICE void merge_pieces(const DecodeArgs &a, size_t row0, int np, int lane) {
+    constexpr int D = C::D, E = D / 32, G = C::G, CH = 2;
+    float M[G], L[G], acc[G][E];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        M[h] = -INFINITY;
+        L[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
+    }
+    for (int p0 = 0; p0 < np; p0 += CH) {
+        float lp[G][CH], ov[G][CH][E];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float *lse = a.ws_lse + (row0 + h) * a.max_parts;
+            const float *op = a.ws_o + (row0 + h) * a.max_parts * D + lane * E;
+#pragma unroll
+            for (int u = 0; u < CH; ++u) {
+                const int p = p0 + u;
+                lp[h][u] = (p < np) ? __ldcg(lse + p) : -INFINITY;
+                if constexpr (E == 4) {
+                    const float4 v = (p < np) ? __ldcg(reinterpret_cast<const float4 *>(op + (size_t)p * D))
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                    ov[h][u][0] = v.x;
+                    ov[h][u][1] = v.y;
+                    ov[h][u][2] = v.z;
+                    ov[h][u][3] = v.w;
+                } else {
+                    const float2 v = (p < np) ? __ldcg(reinterpret_cast<const float2 *>(op + (size_t)p * D))
+                                              : make_float2(0.f, 0.f);
+                    ov[h][u][0] = v.x;
+                    ov[h][u][1] = v.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float mx = M[h];
+#pragma unroll
+            for (int u = 0; u < CH; ++u) mx = fmaxf(mx, lp[h][u]);
+            if (mx == -INFINITY) continue;
+            const float sc = (M[h] == -INFINITY) ? 0.f : ex2(M[h] - mx);
+            M[h] = mx;
+            L[h] *= sc;
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[h][e] *= sc;
+#pragma unroll
+            for (int u = 0; u < CH; ++u) {
+                const float wgt = (lp[h][u] == -INFINITY) ? 0.f : ex2(lp[h][u] - mx);
+                L[h] += wgt;
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[h][e] += wgt * ov[h][u][e];
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float inv = (L[h] > 0.f) ? 1.f / L[h] : 0.f;
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (row0 + h) * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; e += 2)
+            *reinterpret_cast<__nv_bfloat162 *>(out + e) =
+                __floats2bfloat162_rn(acc[h][e] * inv, acc[h][e + 1] * inv);
+    }
+}
+
+// Raw inputs of one item that the consumer loads ahead of time: its q rows
+// (this lane's chunks, head slot h = head h ^ sh) and the fp8 scales.
+template <class C>
+struct QPrefetch {
+    uint4 q[C::G][C::NCH];
+    float ks, vs;
+
+    PA_DEVICE void load(const DecodeArgs &a, const Item &it, const int (&choff)[C::NCH], int sh) {
+        const __nv_bfloat16 *qrow =
+            static_cast<const __nv_bfloat16 *>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.kvh * C::G) * C::D;
+#pragma unroll
+        for (int h = 0; h < C::G; ++h)
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+                q[h][c] = *reinterpret_cast<const uint4 *>(qrow + (h ^ sh) * C::D + choff[c] * 8);
+        ks = C::FP8 ? a.k_scale[it.kvh] : 1.0f;
+        vs = C::FP8 ? a.v_scale[it.kvh] : 1.0f;
+    }
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const DecodeArgs a) {
     constexpr int D = C::D, G = C::G, NW = C::NW, NS = C::NS, VPL = C::VPL, P2 = C::P2, LPT = C::LPT;
     extern __shared__ __align__(128) uint8_t smem[];
     uint8_t *stages = smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::STAGE_BYTES);
     int *stage_valid = reinterpret_cast<int *>(bars + NW * C::NSTAGE);
-    size_t off = C::STAGE_BYTES + (size_t)NW * C::NSTAGE * 12;
-    off = (off + 15) & ~(size_t)15;
-    float *red_acc = reinterpret_cast<float *>(smem + off);  // [NW][G][D]
-    float *red_m = red_acc + NW * G * D;                      // [NW][G]
-    float *red_l = red_m + NW * G;                            // [NW][G]
-    int *s_len = reinterpret_cast<int *>(red_l + NW * G);     // [B]
-    int *s_full = s_len + a.B;                                // [B+1]
-    int *s_tail = s_full + a.B + 1;                           // [B+1]
+    int *wsum = stage_valid + NW * C::NSTAGE;  // [2*NW]
+    int *s_len = wsum + 2 * NW;                // [B]
+    int *s_pre0 = s_len + a.B;                 // [B+1]
+    int *s_pre1 = s_pre0 + a.B + 1;            // [B+1]
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int g = lane / LPT, sub = lane % LPT;
-    const int B = a.B, Hkv = a.Hkv, P = a.partition_tokens;
+    const int B = a.B, Hkv = a.Hkv, P = a.partition_tokens;  // P == 0: balanced split
+    const int gw = blockIdx.x * NW + w, GW = gridDim.x * NW;
 
-    // ---- lengths, then scans of full partitions and tails per sequence
+    // ---- lengths, then exclusive scans over sequences: the balanced split
+    // needs each sequence's offset in the line (Hkv * blocks), the fixed one
+    // the numbers of full partitions and of ragged tails.
     const int cap = a.max_blocks * 16;
     for (int b = tid; b < B; b += C::NT) {
         int len = a.seq_lens[b];
@@ -143,13 +505,14 @@ __global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
     fence_mbar_init();
     __syncthreads();
     {
-        // each thread scans a contiguous run of sequences, then a block scan
-        const int per = (B + C::NT - 1) / C::NT;
+        auto count0 = [&](int len) { return P == 0 ? Hkv * ((len + 15) >> 4) : len / P; };
+        auto count1 = [&](int len) { return P == 0 ? 0 : (int)((len % P) != 0); };
+        const int per = (B + C::NT - 1) / C::NT;  // each thread scans a run of sequences
         const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
         int f = 0, t = 0;
         for (int b = b0; b < b1; ++b) {
-            f += s_len[b] / P;
-            t += (s_len[b] % P) != 0;
+            f += count0(s_len[b]);
+            t += count1(s_len[b]);
         }
         int fi = f, ti = t;  // inclusive warp scan
 #pragma unroll
@@ -160,7 +523,6 @@ __global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
                 ti += tu;
             }
         }
-        int *wsum = reinterpret_cast<int *>(red_acc);  // scratch: 2*NW ints
         if (lane == 31) {
             wsum[w] = fi;
             wsum[NW + w] = ti;
@@ -173,106 +535,47 @@ __global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
         }
         int fx = fb + fi - f, tx = tb + ti - t;  // exclusive prefix of this thread's run
         for (int b = b0; b < b1; ++b) {
-            s_full[b] = fx;
-            s_tail[b] = tx;
-            fx += s_len[b] / P;
-            tx += (s_len[b] % P) != 0;
+            s_pre0[b] = fx;
+            s_pre1[b] = tx;
+            fx += count0(s_len[b]);
+            tx += count1(s_len[b]);
         }
         if (tid == C::NT - 1) {
-            s_full[B] = fx;
-            s_tail[B] = tx;
+            s_pre0[B] = fx;
+            s_pre1[B] = tx;
         }
         __syncthreads();
     }
-    const int NF = s_full[B];
-    const int n_items = (NF + s_tail[B]) * Hkv;
+    Schedule sc;
+    sc.len = s_len;
+    sc.pre0 = s_pre0;
+    sc.pre1 = s_pre1;
+    sc.B = B;
+    sc.Hkv = Hkv;
+    sc.P = P;
+    if (P == 0) {
+        sc.total = s_pre0[B];
+        sc.S = max((sc.total + GW - 1) / GW, kMinShareBlocks);
+        sc.NF = 0;
+    } else {
+        sc.NF = s_pre0[B];
+        sc.total = (sc.NF + s_pre1[B]) * Hkv;
+        sc.S = 0;
+    }
+    // empty sequences produce all-zero rows (no item covers them)
+    for (int b = blockIdx.x; b < B; b += gridDim.x)
+        if (s_len[b] == 0)
+            for (int i = tid; i < a.Hq * D; i += C::NT)
+                static_cast<__nv_bfloat16 *>(a.out)[(size_t)b * a.Hq * D + i] = __float2bfloat16_rn(0.f);
 
-    auto get_item = [&](int i) {
-        Item it;
-        it.kvh = i % Hkv;
-        int u = i / Hkv;
-        if (u < NF) {
-            it.b = upper_index(s_full, B, u);
-            it.part = u - s_full[it.b];
-        } else {
-            u -= NF;
-            it.b = upper_index(s_tail, B, u);
-            it.part = s_full[it.b + 1] - s_full[it.b];
-        }
-        it.len = s_len[it.b];
-        it.nparts = (s_full[it.b + 1] - s_full[it.b]) + (s_tail[it.b + 1] - s_tail[it.b]);
-        const int t0 = it.part * P, t1 = min(t0 + P, it.len);
-        it.blk0 = t0 >> 4;
-        it.nblk = ((t1 + 15) >> 4) - it.blk0;
-        return it;
-    };
-    auto warp_blocks = [&](const Item &it) { return it.nblk > w ? (it.nblk - w + NW - 1) / NW : 0; };
-
-    // ---- producer: one lane issues bulk copies; the warp prefetches table entries
     const uint8_t *kc = static_cast<const uint8_t *>(a.k_cache);
     const uint8_t *vc = static_cast<const uint8_t *>(a.v_cache);
-    auto stage_k = [&](int s) { return stages + ((size_t)(w * C::NSTAGE + s) * 2) * C::BLKB; };
-    auto stage_v = [&](int s) { return stage_k(s) + C::BLKB; };
+    uint8_t *my_stages = stages + (size_t)w * C::NSTAGE * 2 * C::BLKB;
+    uint64_t *my_bars = bars + w * C::NSTAGE;
+    int *my_valid = stage_valid + w * C::NSTAGE;
 
-    auto load_tbl = [&](int item, int &e0, int &e1) {
-        e0 = e1 = -1;
-        if (item >= n_items) return;
-        const Item it = get_item(item);
-        const int nbw = warp_blocks(it);
-        const int32_t *row = a.block_tables + (size_t)it.b * a.max_blocks + it.blk0 + w;
-        if (lane < nbw) e0 = row[NW * lane];
-        if (lane + 32 < nbw) e1 = row[NW * (lane + 32)];
-    };
-
-    int p_item = blockIdx.x, p_j = 0, p_nbw = 0, p_kvh = 0, p_blk0 = 0, p_len = 0;
-    int p_t0, p_t1, n_t0, n_t1;  // table entries of the current and of the next item
-    load_tbl(p_item, p_t0, p_t1);
-    load_tbl(p_item + gridDim.x, n_t0, n_t1);
-    if (p_item < n_items) {
-        const Item it = get_item(p_item);
-        p_nbw = warp_blocks(it);
-        p_kvh = it.kvh;
-        p_blk0 = it.blk0;
-        p_len = it.len;
-    }
-    uint32_t issued = 0, consumed = 0;
-
-    auto produce = [&]() {
-        while (p_item < n_items && p_j >= p_nbw) {
-            p_item += gridDim.x;
-            p_j = 0;
-            p_t0 = n_t0;
-            p_t1 = n_t1;
-            load_tbl(p_item + gridDim.x, n_t0, n_t1);
-            if (p_item < n_items) {
-                const Item it = get_item(p_item);
-                p_nbw = warp_blocks(it);
-                p_kvh = it.kvh;
-                p_blk0 = it.blk0;
-                p_len = it.len;
-            }
-        }
-        if (p_item >= n_items) return;
-        int phys = __shfl_sync(kFull, p_j < 32 ? p_t0 : p_t1, p_j & 31);
-        if (lane == 0) {
-            const int blk = p_blk0 + w + NW * p_j;
-            int valid = min(16, p_len - blk * 16);
-            if (phys < 0 || phys >= a.num_blocks) {
-                flag_error(a.err, PA_DEVERR_BAD_BLOCK);
-                phys = 0;
-                valid = 0;
-            }
-            const int s = issued % C::NSTAGE;
-            stage_valid[w * C::NSTAGE + s] = valid;
-            uint64_t *bar = &bars[w * C::NSTAGE + s];
-            mbar_arrive_expect_tx(bar, 2 * C::BLKB);
-            const size_t src = ((size_t)phys * Hkv + p_kvh) * C::BLKB;
-            bulk_g2s(stage_k(s), kc + src, C::BLKB, bar);
-            bulk_g2s(stage_v(s), vc + src, C::BLKB, bar);
-        }
-        ++issued;
-        ++p_j;
-    };
+    Producer<C> prod;
+    prod.init(sc, a, gw, GW, lane);
 
     // ---- per-lane constants: which 16-byte chunks of a row this lane reads.
     // Odd token groups visit their chunks in the other order so that lanes
@@ -280,87 +583,61 @@ __global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
     int choff[C::NCH];
 #pragma unroll
     for (int c = 0; c < C::NCH; ++c) choff[c] = sub + LPT * ((c + g) % C::NCH);
+    // register layout of the partial scores (see rs_level)
+    const int S = C::RS ? sub * VPL : 0;
+    const int sh = S % G;  // head slot h holds head h ^ sh
+    const int sj = S / G;  // token slot j reads token j ^ sj of the sub-step
+    uint32_t consumed = 0;
 
-    auto load_row = [&](const uint8_t *row, float2 (&f)[P2]) {
-#pragma unroll
-        for (int c = 0; c < C::NCH; ++c) {
-            if constexpr (!C::FP8) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(row + choff[c] * C::CHB);
-                f[4 * c + 0] = bf16x2_to_float2(u.x);
-                f[4 * c + 1] = bf16x2_to_float2(u.y);
-                f[4 * c + 2] = bf16x2_to_float2(u.z);
-                f[4 * c + 3] = bf16x2_to_float2(u.w);
-            } else {
-                const uint2 u = *reinterpret_cast<const uint2 *>(row + choff[c] * C::CHB);
-                f[4 * c + 0] = e4m3x2_to_float2((uint16_t)(u.x & 0xffff));
-                f[4 * c + 1] = e4m3x2_to_float2((uint16_t)(u.x >> 16));
-                f[4 * c + 2] = e4m3x2_to_float2((uint16_t)(u.y & 0xffff));
-                f[4 * c + 3] = e4m3x2_to_float2((uint16_t)(u.y >> 16));
-            }
-        }
-    };
+    for (int prime = 0; prime < C::NSTAGE; ++prime) prod.produce(sc, a, lane, kc, vc, my_stages, my_bars, my_valid);
 
-    // scores this lane owns after the reduction: sub-step token j and head h
-    int own_j[VPL], own_h[VPL];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-        const int idx = (C::RS ? sub * VPL : 0) + i;
-        own_j[i] = idx / G;
-        own_h[i] = idx % G;
-    }
+    ItemIter items;
+    items.start(sc, gw, GW);
+    Item it, nx;
+    bool have = items.next(sc, it);
+    bool have_nx = have && items.next(sc, nx);
+    QPrefetch<C> qp;
+    if (have) qp.load(a, it, choff, sh);
+    while (have) {
+        const float vscale = qp.vs;
+        const float qs = a.scale * kLog2e * qp.ks;
+        const size_t row0 = (size_t)it.b * a.Hq + (size_t)it.kvh * G;  // first q head of the group
 
-    for (int prime = 0; prime < C::NSTAGE; ++prime) produce();
-
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const Item it = get_item(item);
-        const int nbw = warp_blocks(it);
-        const float kscale = C::FP8 ? a.k_scale[it.kvh] : 1.0f;
-        const float vscale = C::FP8 ? a.v_scale[it.kvh] : 1.0f;
-        const float qs = a.scale * kLog2e * kscale;
-
+        // q of the GQA group in fp32, pre-scaled into log2 units; slot h = head h ^ sh
         float2 q2[G][P2], acc2[G][P2];
-        float m[G], m_own[VPL], l_own[VPL];
-        {
-            const __nv_bfloat16 *qrow =
-                static_cast<const __nv_bfloat16 *>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.kvh * G) * D;
+        float m[G], l[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < G; ++h) {
 #pragma unroll
-                for (int c = 0; c < C::NCH; ++c) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(qrow + h * D + choff[c] * 8);
-                    const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
+            for (int c = 0; c < C::NCH; ++c) {
+                const uint32_t ws[4] = {qp.q[h][c].x, qp.q[h][c].y, qp.q[h][c].z, qp.q[h][c].w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = bf16x2_to_float2(ws[e]);
-                        q2[h][4 * c + e] = make_float2(f.x * qs, f.y * qs);
-                        acc2[h][4 * c + e] = make_float2(0.f, 0.f);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = bf16x2_to_float2(ws[e]);
+                    q2[h][4 * c + e] = make_float2(f.x * qs, f.y * qs);
+                    acc2[h][4 * c + e] = make_float2(0.f, 0.f);
                 }
-                m[h] = -INFINITY;
             }
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                m_own[i] = -INFINITY;
-                l_own[i] = 0.f;
-            }
+            m[h] = -INFINITY;
+            l[h] = 0.f;
         }
 
-        for (int j = 0; j < nbw; ++j) {
+        for (int j = 0; j < it.nblk; ++j) {
             const int s = consumed % C::NSTAGE;
-            if (!mbar_wait(&bars[w * C::NSTAGE + s], (consumed / C::NSTAGE) & 1) && lane == 0)
+            if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
                 flag_error(a.err, PA_DEVERR_TIMEOUT);
-            const int valid = stage_valid[w * C::NSTAGE + s];
-            const uint8_t *Kb = stage_k(s), *Vb = stage_v(s);
+            const int valid = my_valid[s];
+            const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
 
 #pragma unroll
             for (int sb = 0; sb < C::NSUB; ++sb) {
-                // --- q . k for this group's TSUB tokens, all G heads
+                const int t_base = g + C::NGRP * sb * C::TSUB;
+                // --- q . k: partial dot products over this lane's dims
                 float part[NS];
 #pragma unroll
                 for (int jj = 0; jj < C::TSUB; ++jj) {
-                    const int t = g + C::NGRP * (sb * C::TSUB + jj);
                     float2 kf[P2];
-                    load_row(Kb + t * C::ROWB, kf);
+                    load_row<C>(Kb + (t_base + C::NGRP * (jj ^ sj)) * C::ROWB, choff, kf);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         float2 d2 = make_float2(0.f, 0.f);
@@ -369,104 +646,55 @@ __global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
                         part[jj * G + h] = d2.x + d2.y;
                     }
                 }
-                // --- combine partial dot products across the LPT lanes of the group
-                if constexpr (C::RS) {
-                    int n = NS;
-#pragma unroll
-                    for (int mask = LPT / 2; mask >= 1; mask >>= 1) {
-                        n >>= 1;
-                        const bool hi = (sub & mask) != 0;
-#pragma unroll
-                        for (int k = 0; k < NS / 2; ++k) {
-                            if (k < n) {
-                                const float send = hi ? part[k] : part[k + n];
-                                const float keep = hi ? part[k + n] : part[k];
-                                part[k] = keep + __shfl_xor_sync(kFull, send, mask);
-                            }
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int mask = LPT / 2; mask >= 1; mask >>= 1)
-#pragma unroll
-                        for (int k = 0; k < NS; ++k) part[k] += __shfl_xor_sync(kFull, part[k], mask);
-                }
-                // --- mask tokens past the end, check whether the running max must move
-                float sc[VPL];
+                // --- complete the scores across the LPT lanes of the group
+                if constexpr (C::RS)
+                    rs_level<LPT / 2, NS / 2, NS>(part);
+                else
+                    allreduce_level<LPT / 2, NS>(part);
+                // --- owned score i: head slot i % G, token slot i / G.
+                // Mask tokens past the end; move the running max only when a
+                // score exceeds it by more than the threshold.
+                float sco[VPL];
                 bool need = false;
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
-                    const int t = g + C::NGRP * (sb * C::TSUB + own_j[i]);
-                    sc[i] = (t < valid) ? part[i] : -INFINITY;
-                    need |= sc[i] > m_own[i] + kRescaleThreshold;
+                    const int t = t_base + C::NGRP * ((i / G) ^ sj);
+                    sco[i] = (t < valid) ? part[i] : -INFINITY;
+                    need |= sco[i] > m[i % G] + kRescaleThreshold;
                 }
                 if (__any_sync(kFull, need)) {
                     float bm[G];
 #pragma unroll
                     for (int h = 0; h < G; ++h) bm[h] = -INFINITY;
 #pragma unroll
-                    for (int i = 0; i < VPL; ++i)
-#pragma unroll
-                        for (int h = 0; h < G; ++h)
-                            if (own_h[i] == h) bm[h] = fmaxf(bm[h], sc[i]);
-                    if constexpr (C::RS) {
-#pragma unroll
-                        for (int mask = LPT / 2; mask >= 1; mask >>= 1)
-#pragma unroll
-                            for (int h = 0; h < G; ++h) bm[h] = fmaxf(bm[h], __shfl_xor_sync(kFull, bm[h], mask));
-                    }
-                    float alpha[G];
+                    for (int i = 0; i < VPL; ++i) bm[i % G] = fmaxf(bm[i % G], sco[i]);
+                    if constexpr (C::RS) perm_allreduce<LPT / 2, VPL, G, true>(bm);
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         const float mn = fmaxf(m[h], bm[h]);
-                        alpha[h] = (mn == -INFINITY) ? 1.f : ex2(m[h] - mn);
+                        const float alpha = (mn == -INFINITY) ? 1.f : ex2(m[h] - mn);
                         m[h] = mn;
+                        l[h] *= alpha;
 #pragma unroll
-                        for (int k = 0; k < P2; ++k)
-                            acc2[h][k] = fmul2(acc2[h][k], make_float2(alpha[h], alpha[h]));
-                    }
-#pragma unroll
-                    for (int i = 0; i < VPL; ++i) {
-#pragma unroll
-                        for (int h = 0; h < G; ++h)
-                            if (own_h[i] == h) {
-                                l_own[i] *= alpha[h];
-                                m_own[i] = m[h];
-                            }
+                        for (int k = 0; k < P2; ++k) acc2[h][k] = fmul2(acc2[h][k], make_float2(alpha, alpha));
                     }
                 }
                 // --- probabilities of the owned scores, then all-gather them
                 float pr[NS];
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
-                    const float p = (sc[i] == -INFINITY) ? 0.f : ex2(sc[i] - m_own[i]);
-                    l_own[i] += p;
+                    const float p = (sco[i] == -INFINITY) ? 0.f : ex2(sco[i] - m[i % G]);
+                    l[i % G] += p;
                     pr[i] = p;
                 }
-                if constexpr (C::RS) {
-                    int n = VPL;
-#pragma unroll
-                    for (int mask = 1; mask < LPT; mask <<= 1) {
-                        const bool hi = (sub & mask) != 0;
-#pragma unroll
-                        for (int k = 0; k < NS / 2; ++k) {
-                            if (k < n) {
-                                const float r = __shfl_xor_sync(kFull, pr[k], mask);
-                                const float mine = pr[k];
-                                pr[k] = hi ? r : mine;
-                                pr[k + n] = hi ? mine : r;
-                            }
-                        }
-                        n <<= 1;
-                    }
-                }
-                // --- acc += p * v for this group's tokens
+                if constexpr (C::RS) ag_level<1, LPT, VPL, NS>(pr);
+                // --- acc += p * v over this group's tokens
 #pragma unroll
                 for (int jj = 0; jj < C::TSUB; ++jj) {
-                    const int t = g + C::NGRP * (sb * C::TSUB + jj);
+                    const int t = t_base + C::NGRP * (jj ^ sj);
                     if (t < valid) {
                         float2 vf[P2];
-                        load_row(Vb + t * C::ROWB, vf);
+                        load_row<C>(Vb + t * C::ROWB, choff, vf);
 #pragma unroll
                         for (int h = 0; h < G; ++h) {
                             const float p = pr[jj * G + h];
@@ -479,179 +707,124 @@ __global__ void __launch_bounds__(C::NT) decode_kernel(const DecodeArgs a) {
             }
             __syncwarp();
             ++consumed;
-            produce();
+            prod.produce(sc, a, lane, kc, vc, my_stages, my_bars, my_valid);
         }
 
-        // ---- epilogue: normaliser per head within the group
-        float l[G];
+        // ---- the next item's q and scales are needed right after this
+        // epilogue: start their loads now so the latency overlaps it
+        if (have_nx) qp.load(a, nx, choff, sh);
+
+        // ---- epilogue: complete the normaliser per head across the group,
+        // then merge the token groups (same dims, different tokens)
+        if constexpr (C::RS) perm_allreduce<LPT / 2, VPL, G, false>(l);
+        group_merge<LPT, LPT, G, P2, C::NCH == 2>(m, l, acc2);
+
+        // every group now holds the warp's result; group 0 writes it
+        if (it.npieces == 1) {
+            if (g == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            l[h] = 0.f;
+                for (int h = 0; h < G; ++h) {
+                    const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + (row0 + (h ^ sh)) * D;
 #pragma unroll
-            for (int i = 0; i < VPL; ++i)
-                if (own_h[i] == h) l[h] += l_own[i];
-        }
-        if constexpr (C::RS) {
+                    for (int c = 0; c < C::NCH; ++c) {
+                        uint32_t wds[4];
 #pragma unroll
-            for (int mask = 1; mask < LPT; mask <<= 1)
-#pragma unroll
-                for (int h = 0; h < G; ++h) l[h] += __shfl_xor_sync(kFull, l[h], mask);
-        }
-        // ---- combine token groups of this warp (same dims, different tokens)
-#pragma unroll
-        for (int mask = LPT; mask < 32; mask <<= 1) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float mo = __shfl_xor_sync(kFull, m[h], mask);
-                const float lo = __shfl_xor_sync(kFull, l[h], mask);
-                const float M = fmaxf(m[h], mo);
-                const float am = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - M);
-                const float ao = (mo == -INFINITY) ? 0.f : ex2(mo - M);
-                l[h] = l[h] * am + lo * ao;
-                m[h] = M;
-                // Groups of opposite parity visit their chunks in swapped
-                // order: pull the partner's register that holds my chunk.
-                constexpr bool swap = (C::NCH == 2);
-                float2 rx[P2];
-#pragma unroll
-                for (int k = 0; k < P2; ++k) {
-                    const int ks = (swap && mask == LPT) ? (k ^ 4) : k;
-                    rx[k].x = __shfl_xor_sync(kFull, acc2[h][ks].x, mask);
-                    rx[k].y = __shfl_xor_sync(kFull, acc2[h][ks].y, mask);
-                }
-#pragma unroll
-                for (int k = 0; k < P2; ++k)
-                    acc2[h][k] = ffma2(acc2[h][k], make_float2(am, am), make_float2(rx[k].x * ao, rx[k].y * ao));
-            }
-        }
-        // ---- combine warps through shared memory
-        if (g == 0) {
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-#pragma unroll
-                for (int c = 0; c < C::NCH; ++c) {
-                    float *dst = red_acc + ((size_t)w * G + h) * D + choff[c] * 8;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        dst[2 * e] = acc2[h][4 * c + e].x;
-                        dst[2 * e + 1] = acc2[h][4 * c + e].y;
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 bb =
+                                __floats2bfloat162_rn(acc2[h][4 * c + e].x * inv, acc2[h][4 * c + e].y * inv);
+                            wds[e] = *reinterpret_cast<const uint32_t *>(&bb);
+                        }
+                        *reinterpret_cast<uint4 *>(dst + choff[c] * 8) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
                     }
                 }
-                if (sub == 0) {
-                    red_m[w * G + h] = m[h];
-                    red_l[w * G + h] = l[h];
+            }
+        } else {
+            // ---- split-K: write this piece, count it; the warp completing
+            // the last piece of this (sequence, kv head) merges them all
+            if (g == 0) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
+                    float *dst = a.ws_o + ((row0 + (h ^ sh)) * a.max_parts + it.piece) * D;
+#pragma unroll
+                    for (int c = 0; c < C::NCH; ++c) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + choff[c] * 8);
+                        d4[0] = make_float4(acc2[h][4 * c].x * inv, acc2[h][4 * c].y * inv,
+                                            acc2[h][4 * c + 1].x * inv, acc2[h][4 * c + 1].y * inv);
+                        d4[1] = make_float4(acc2[h][4 * c + 2].x * inv, acc2[h][4 * c + 2].y * inv,
+                                            acc2[h][4 * c + 3].x * inv, acc2[h][4 * c + 3].y * inv);
+                    }
+                    if (sub == 0)  // sub 0 has sh == 0: slot h is head h
+                        a.ws_lse[(row0 + h) * a.max_parts + it.piece] = (l[h] > 0.f) ? m[h] + lg2(l[h]) : -INFINITY;
                 }
+                __threadfence();
+            }
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) {
+                int *ctr = a.counters + (size_t)it.b * Hkv + it.kvh;
+                last = atomicAdd(ctr, 1) == it.npieces - 1;
+                if (last) *ctr = 0;  // every piece has arrived: ready for the next call
+            }
+            last = __shfl_sync(kFull, last, 0);
+            if (last) {
+                __threadfence();
+                merge_pieces<C>(a, row0, it.npieces, lane);
             }
         }
-        __syncthreads();
-        const bool single = it.nparts == 1;
-        for (int idx = tid; idx < G * D; idx += C::NT) {
-            const int h = idx / D, d = idx % D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int v = 0; v < NW; ++v) M = fmaxf(M, red_m[v * G + h]);
-            float L = 0.f, O = 0.f;
-#pragma unroll
-            for (int v = 0; v < NW; ++v) {
-                const float mv = red_m[v * G + h];
-                const float f = (mv == -INFINITY) ? 0.f : ex2(mv - M);
-                L += red_l[v * G + h] * f;
-                O += red_acc[((size_t)v * G + h) * D + d] * f;
-            }
-            const float o = (L > 0.f) ? (O / L) * vscale : 0.f;
-            const size_t row = (size_t)it.b * a.Hq + (size_t)it.kvh * G + h;
-            if (single) {
-                static_cast<__nv_bfloat16 *>(a.out)[row * D + d] = __float2bfloat16_rn(o);
-            } else {
-                a.ws_o[(row * a.max_parts + it.part) * D + d] = o;
-                if (d == 0) a.ws_lse[row * a.max_parts + it.part] = (L > 0.f) ? M + lg2(L) : -INFINITY;
-            }
-        }
-        __syncthreads();
+        it = nx;
+        have = have_nx;
+        have_nx = have && items.next(sc, nx);
     }
-}
-
-// One warp per (sequence, query head): log-sum-exp merge of the partials of
-// sequences with more than one partition; zero rows for empty sequences.
-template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
-    constexpr int E = D / 32;  // dims per lane
-    const int b = blockIdx.x, h = blockIdx.y * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (h >= a.Hq) return;
-    int len = a.seq_lens[b];
-    if (len < 0 || len > a.max_blocks * 16) len = 0;
-    const int P = a.partition_tokens;
-    const int nparts = (len + P - 1) / P;
-    if (nparts == 1) return;
-    const size_t row = (size_t)b * a.Hq + h;
-    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + row * D + lane * E;
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    if (nparts > 1) {
-        const float *lse = a.ws_lse + row * a.max_parts;
-        const float *o = a.ws_o + row * a.max_parts * D + lane * E;
-        float M = -INFINITY;
-        for (int p = lane; p < nparts; p += 32) M = fmaxf(M, lse[p]);
-#pragma unroll
-        for (int mask = 16; mask >= 1; mask >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, mask));
-        float L = 0.f;
-        for (int p = 0; p < nparts; ++p) {
-            const float lp = lse[p];
-            const float wgt = (lp == -INFINITY) ? 0.f : ex2(lp - M);
-            L += wgt;
-            if constexpr (E == 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(o + (size_t)p * D);
-                acc[0] += wgt * v.x;
-                acc[1] += wgt * v.y;
-                acc[2] += wgt * v.z;
-                acc[3] += wgt * v.w;
-            } else {
-                const float2 v = *reinterpret_cast<const float2 *>(o + (size_t)p * D);
-                acc[0] += wgt * v.x;
-                acc[1] += wgt * v.y;
-            }
-        }
-        const float inv = (L > 0.f) ? 1.f / L : 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] *= inv;
-    }
-#pragma unroll
-    for (int e = 0; e < E; e += 2)
-        *reinterpret_cast<__nv_bfloat162 *>(out + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
 }
 
 template <class C>
 cudaError_t run(const DecodeArgs &a, cudaStream_t st) {
-    // Opt in to the large dynamic shared-memory carve-out once per device.
+    // Per device: opt in to the large shared-memory carve-out once, and
+    // remember SM count and occupancy per shared-memory size (B decides it).
+    struct Occ {
+        int smem_key = -1, ctas = 0;
+    };
     static std::mutex mu;
     static bool ready[64] = {};
-    int dev = 0, sms = 0, occ = 0;
+    static int sms[64] = {};
+    static Occ occ[64][4];
+    int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const size_t smem = smem_bytes<C>(a.B);
+    int ctas = 0;
     {
         std::lock_guard<std::mutex> lock(mu);
         if (!ready[dev]) {
             e = cudaFuncSetAttribute(decode_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem_bytes<C>(2048));
+                                     (int)smem_bytes<C>(kMaxDecodeSeqs));
+            if (e != cudaSuccess) return e;
+            e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
             if (e != cudaSuccess) return e;
             ready[dev] = true;
         }
+        Occ *slot = nullptr;
+        for (auto &o : occ[dev])
+            if (o.smem_key == (int)smem) slot = &o;
+        if (!slot) {
+            int n = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<C>, C::NT, smem);
+            if (e != cudaSuccess) return e;
+            slot = &occ[dev][(smem / 16) % 4];
+            slot->smem_key = (int)smem;
+            slot->ctas = n < 1 ? 1 : n;
+        }
+        ctas = slot->ctas * sms[dev];
     }
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    const size_t smem = smem_bytes<C>(a.B);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<C>, C::NT, smem);
-    if (e != cudaSuccess) return e;
-    if (occ < 1) occ = 1;
-    const long long upper = (long long)a.Hkv * a.B * a.max_parts;
-    const long long grid = std::min<long long>(upper, (long long)sms * occ);
-    if (grid > 0) decode_kernel<C><<<(unsigned)grid, C::NT, smem, st>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    dim3 mgrid(a.B, (a.Hq + 3) / 4);
-    merge_kernel<C::D><<<mgrid, 128, 0, st>>>(a);
+    // enough CTAs to cover every warp-sized unit of work, at most one wave
+    const long long units = a.partition_tokens == 0
+                                ? (long long)a.Hkv * a.B * a.max_blocks / kMinShareBlocks + 1
+                                : (long long)a.Hkv * a.B * a.max_parts;
+    const long long grid = std::max<long long>(1, std::min<long long>((units + C::NW - 1) / C::NW, ctas));
+    decode_kernel<C><<<(unsigned)grid, C::NT, smem, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -668,6 +841,8 @@ cudaError_t by_group(const DecodeArgs &a, cudaStream_t st) {
 
 }  // namespace
 
+size_t decode_ws_counter_bytes() { return (size_t)kMaxDecodeSeqs * kMaxDecodeKvHeads * sizeof(int); }
+
 size_t decode_ws_o_bytes(int B, int Hq, int D, int max_parts) {
     const size_t o = (size_t)B * Hq * max_parts * D * sizeof(float);
     return (o + 255) & ~(size_t)255;
@@ -675,7 +850,7 @@ size_t decode_ws_o_bytes(int B, int Hq, int D, int max_parts) {
 
 size_t decode_ws_bytes(int B, int Hq, int D, int max_parts) {
     const size_t lse = (size_t)B * Hq * max_parts * sizeof(float);
-    return decode_ws_o_bytes(B, Hq, D, max_parts) + ((lse + 255) & ~(size_t)255);
+    return decode_ws_counter_bytes() + decode_ws_o_bytes(B, Hq, D, max_parts) + ((lse + 255) & ~(size_t)255);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {

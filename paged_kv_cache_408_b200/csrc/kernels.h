@@ -39,8 +39,9 @@ struct DecodeArgs {
     int64_t num_blocks;
     float scale;
     const float *k_scale, *v_scale;
-    int partition_tokens;  // multiple of 16
-    int max_parts;         // partitions of the longest possible sequence
+    int partition_tokens;  // 0: balanced split; else a multiple of 16 (fixed partitions)
+    int max_parts;         // most pieces one (sequence, kv head) can be cut into
+    int *counters;         // [kMaxDecodeSeqs * kMaxDecodeKvHeads] arrivals per (seq, kv head); zero between calls
     float *ws_o;           // [B][Hq][max_parts][D]
     float *ws_lse;         // [B][Hq][max_parts]
     bool fp8;
@@ -64,7 +65,20 @@ cudaError_t launch_copy_blocks(const CopyArgs &a, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
 
-// Workspace layout shared by pa_decode_workspace_size and pa_decode.
+// Workspace layout shared by pa_decode_workspace_size and pa_decode:
+// [arrival counters | partial outputs | partial log2-sum-exp].  The counter
+// region has a fixed size so it never overlaps data of a call with another
+// batch size; it must be zero before the first call and every call leaves it
+// zero.
+constexpr int kMaxDecodeSeqs = 2048;
+constexpr int kMinShareBlocks = 16;  // balanced split: smallest per-CTA share, in blocks
+constexpr int kMaxDecodeKvHeads = 128;
+size_t decode_ws_counter_bytes();
+// Pieces one (sequence, kv head) of max_blocks blocks can be cut into.
+inline int decode_max_parts(int max_blocks, int partition_tokens) {
+    return partition_tokens == 0 ? max_blocks / kMinShareBlocks + 2
+                                 : (max_blocks * 16 + partition_tokens - 1) / partition_tokens;
+}
 size_t decode_ws_o_bytes(int B, int Hq, int D, int max_parts);
 size_t decode_ws_bytes(int B, int Hq, int D, int max_parts);
 

@@ -169,9 +169,10 @@ def decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, p
 
 
 def alloc_workspace(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, partition_tokens=0, device=None):
-    """Caller-side helper: a torch buffer large enough for pa_decode."""
+    """Caller-side helper: a zero-filled torch buffer large enough for
+    pa_decode (the library needs it zeroed once; calls keep it that way)."""
     n = decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, partition_tokens)
-    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
 def decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale=None, v_scale=None, workspace=None,

@@ -71,15 +71,17 @@ def test_decode_zero_length_rows_are_zero(cuda_device):
         assert_attn_close(out, oracle_decode(c), "zero-length rows")
 
 
-def test_decode_is_batch_invariant(cuda_device):
-    """A sequence's output does not depend on what else is in the batch."""
+@pytest.mark.parametrize("part", [16, 256, 1024])
+def test_fixed_partitions_are_batch_invariant(cuda_device, part):
+    """With fixed partitions a sequence's output is bitwise independent of
+    what else is in the batch."""
     c = I.make_decode_case(8, [700, 33, 1500, 5, 260], 32, 8, 128)
     kc, vc = cache_to_device(c)
-    full = host_bits(run_decode(c, kc, vc))
+    full = host_bits(run_decode(c, kc, vc, partition_tokens=part))
     for rows in ([2], [4, 2, 0], [1, 3]):
         rows = np.array(rows)
         sub = host_bits(run_decode(c, kc, vc, seq_lens=c.seq_lens[rows], block_tables=c.block_tables[rows],
-                                   q=c.q[rows]))
+                                   q=c.q[rows], partition_tokens=part))
         assert np.array_equal(sub, full[rows])
 
 
@@ -173,3 +175,22 @@ def test_bad_slot_and_bad_length_are_flagged(cuda_device):
     lens[2] = 10_000  # longer than the block table
     run_decode(c, kc, vc, seq_lens=lens)
     assert ops.get_last_device_error() & ops.DEVERR_BAD_LEN
+
+
+@pytest.mark.parametrize("part", [0, 256])
+def test_workspace_reuse_across_calls_and_batch_sizes(cuda_device, part):
+    """One zero-filled workspace serves calls of any batch size; the merge's
+    arrival counters (its first MiB) are back at zero after every call."""
+    c = I.make_decode_case(15, [1000, 40, 2048, 513, 300], 32, 8, 128)
+    kc, vc = cache_to_device(c)
+    ws = ops.alloc_workspace(64, 32, 128, c.block_tables.shape[1], part, device=kc.device)
+    ref = oracle_decode(c)
+    for rows in ([0, 1, 2, 3, 4], [2], [3, 0], [4, 2, 1], [0, 1, 2, 3, 4]):
+        rows = np.array(rows)
+        qd = dev_bf16(c.q[rows])
+        out = torch.empty_like(qd)
+        ops.decode(out, qd, kc, vc, dev(c.block_tables[rows], np.int32), dev(c.seq_lens[rows], np.int32), c.scale,
+                   workspace=ws, partition_tokens=part)
+        torch.cuda.synchronize()
+        assert_attn_close(to_float(out), ref[rows], f"rows {rows.tolist()}")
+        assert int(ws[:1 << 20].count_nonzero()) == 0
