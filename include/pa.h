@@ -213,6 +213,41 @@ int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const i
                      const float *k_scale, const float *v_scale, const pa_cache_desc *desc, pa_stream_t stream);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  There is no counterpart of this entry point in the source pages.
+ *
+ * Some callers cannot call cudaMalloc: a plugin hosted by a serving engine
+ * whose memory pool has already claimed the device (engines typically
+ * reserve nearly all HBM for the KV cache at start-up, so a late cudaMalloc
+ * fails or fragments the pool), or an integration that must not trigger the
+ * implicit device synchronisation cudaMalloc/cudaFree can cause.  This
+ * variant takes the same arguments as pa_decode minus the workspace: its
+ * split-K scratch lives in a fixed device array inside libpa.so,
+ * PA_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) large, which every GPU that loads
+ * the library holds until the process exits.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ *
+ *   - A shape whose pa_decode_workspace_size() exceeds the array returns
+ *     PA_ERR_WORKSPACE before anything is enqueued (use pa_decode with a
+ *     caller workspace, or fixed partitions, which need less scratch).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, once per device, with that device current);
+ *     make that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents; each call first clears (cudaMemsetAsync on `stream`)
+ *     the part that must start at zero.  Calls that overlap on the GPU (on
+ *     different streams without ordering) race on the array and give wrong
+ *     results: order them.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int pa_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *seq_lens, int32_t num_seqs,
+                      int32_t max_blocks_per_seq, int32_t num_q_heads, float scale, const float *k_scale,
+                      const float *v_scale, int32_t partition_tokens, const pa_cache_desc *desc,
+                      pa_stream_t stream);
+
+/*
  * pa_get_last_device_error -- synchronise `stream`, return the device status
  * word (PA_DEVERR_* bits, 0 if clean) in *flags and clear it.  Returns
  * PA_ERR_DEVICE if any bit was set, PA_OK otherwise.

@@ -58,6 +58,8 @@ int resolve_partition(int32_t partition_tokens, int *out) {
 
 }  // namespace
 
+unsigned *pa::status_word() { return status_word_ptr(); }
+
 extern "C" {
 
 int pa_version(void) { return 100; }

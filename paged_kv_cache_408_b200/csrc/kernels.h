@@ -65,6 +65,9 @@ cudaError_t launch_copy_blocks(const CopyArgs &a, cudaStream_t st);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
 
+// Device address of the status word on the current device (nullptr if unknown).
+unsigned *status_word();
+
 // Workspace layout shared by pa_decode_workspace_size and pa_decode:
 // [arrival counters | partial outputs | partial log2-sum-exp].  The counter
 // region has a fixed size so it never overlaps data of a call with another

@@ -24,7 +24,7 @@ DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_LEN, DEVERR_BAD_PAIR, DEVERR_TIMEO
 
 EXPORTED = (
     "pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_size", "pa_decode", "pa_prefill_chunk",
-    "pa_get_last_device_error", "pa_status_string", "pa_version",
+    "pa_get_last_device_error", "pa_status_string", "pa_version", "pa_decode_noalloc",
 )
 
 
@@ -57,6 +57,7 @@ def lib():
         L.pa_decode.argtypes = [p, p, p, p, p, p, i32, i32, i32, f32, p, p, i32, p, sz, C.POINTER(CacheDesc), p]
         L.pa_prefill_chunk.argtypes = [p, p, p, p, p, i32, i32, i32, i32, p, p, f32, p, p, C.POINTER(CacheDesc), p]
         L.pa_get_last_device_error.argtypes = [C.POINTER(C.c_uint32), p]
+        L.pa_decode_noalloc.argtypes = [p, p, p, p, p, p, i32, i32, i32, f32, p, p, i32, C.POINTER(CacheDesc), p]
         L.pa_status_string.argtypes = [C.c_int]
         L.pa_status_string.restype = C.c_char_p
         for f in EXPORTED:
@@ -200,6 +201,30 @@ def decode(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale=None
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), B,
         block_tables.shape[1], Hq, float(scale), _ptr(ks), _ptr(vs), int(partition_tokens), _ptr(workspace),
         ws_bytes, C.byref(desc), _stream(stream)))
+
+
+def decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_scale=None, v_scale=None,
+                   partition_tokens=0, stream=None):
+    """pa_decode_noalloc: pa_decode without a caller workspace, for callers
+    that cannot allocate device memory; the library's fixed 16 MiB scratch is
+    used instead (shapes that need more raise PAError with
+    PA_ERR_WORKSPACE).  Calls must not overlap on the GPU."""
+    desc = _caches(k_cache, v_cache)
+    dev = k_cache.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    B, Hq, D = q.shape
+    if out.shape != q.shape or D != desc.head_dim:
+        raise ValueError("out/q shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and seq_lens [B]")
+    ks, vs = _scales(desc, k_scale, v_scale, dev)
+    _check("pa_decode_noalloc", lib().pa_decode_noalloc(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), B,
+        block_tables.shape[1], Hq, float(scale), _ptr(ks), _ptr(vs), int(partition_tokens), C.byref(desc),
+        _stream(stream)))
 
 
 def prefill_chunk(out, q, cu_q_lens, prefix_lens, block_tables, k_cache, v_cache, scale, max_q_len,
