@@ -204,12 +204,16 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
  *                 and attends keys 0..prefix_lens[c]+i inclusive.
  *   block_tables  int32 [num_chunks][max_blocks_per_seq].
  *   max_q_len     host upper bound on any chunk's length (sizes the grid).
+ *   total_q_tokens  rows of q and out (= cu_q_lens[num_chunks]); chunks
+ *                 reaching past it are rejected on the device.
  * The chunk's own K/V must already be in the cache (pa_write_kv first).
- * bf16 cache only; an fp8 cache returns PA_ERR_UNSUPPORTED.
+ * bf16 cache only; an fp8 cache returns PA_ERR_UNSUPPORTED.  head_dim 64 or
+ * 128; num_q_heads / num_kv_heads in {1,2,4,8}.
  */
 int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const int32_t *prefix_lens,
                      const int32_t *block_tables, int32_t num_chunks, int32_t max_blocks_per_seq,
-                     int32_t num_q_heads, int32_t max_q_len, const void *k_cache, const void *v_cache, float scale,
+                     int32_t num_q_heads, int32_t max_q_len, int32_t total_q_tokens, const void *k_cache,
+                     const void *v_cache, float scale,
                      const float *k_scale, const float *v_scale, const pa_cache_desc *desc, pa_stream_t stream);
 
 /*

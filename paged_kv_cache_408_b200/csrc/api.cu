@@ -159,21 +159,25 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
 
 int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const int32_t *prefix_lens,
                      const int32_t *block_tables, int32_t num_chunks, int32_t max_blocks_per_seq,
-                     int32_t num_q_heads, int32_t max_q_len, const void *k_cache, const void *v_cache, float scale,
-                     const float *k_scale, const float *v_scale, const pa_cache_desc *desc, pa_stream_t stream) {
+                     int32_t num_q_heads, int32_t max_q_len, int32_t total_q_tokens, const void *k_cache,
+                     const void *v_cache, float scale, const float *k_scale, const float *v_scale,
+                     const pa_cache_desc *desc, pa_stream_t stream) {
     (void)k_scale;
     (void)v_scale;
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
-    if (num_chunks < 0 || max_blocks_per_seq <= 0 || num_q_heads <= 0 || max_q_len < 0) return PA_ERR_INVALID_ARG;
+    if (num_chunks < 0 || max_blocks_per_seq <= 0 || num_q_heads <= 0 || max_q_len < 0 || total_q_tokens < 0)
+        return PA_ERR_INVALID_ARG;
     if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    const int G = num_q_heads / desc->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
     if (desc->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
-    if (num_chunks == 0 || max_q_len == 0) return PA_OK;
+    if (num_chunks == 0 || max_q_len == 0 || total_q_tokens == 0) return PA_OK;
     if (!out || !q || !cu_q_lens || !prefix_lens || !block_tables || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
     pa::PrefillArgs a{out, q, cu_q_lens, prefix_lens, block_tables, num_chunks, max_blocks_per_seq, num_q_heads,
-                      desc->num_kv_heads, desc->head_dim, max_q_len, 0, desc->num_blocks, k_cache, v_cache, scale,
-                      status_word_ptr()};
+                      desc->num_kv_heads, desc->head_dim, max_q_len, total_q_tokens, desc->num_blocks, k_cache,
+                      v_cache, scale, status_word_ptr()};
     return from_cuda(pa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 

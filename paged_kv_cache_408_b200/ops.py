@@ -55,7 +55,8 @@ def lib():
         L.pa_copy_blocks.argtypes = [p, p, p, i32, C.POINTER(CacheDesc), p]
         L.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, C.POINTER(sz)]
         L.pa_decode.argtypes = [p, p, p, p, p, p, i32, i32, i32, f32, p, p, i32, p, sz, C.POINTER(CacheDesc), p]
-        L.pa_prefill_chunk.argtypes = [p, p, p, p, p, i32, i32, i32, i32, p, p, f32, p, p, C.POINTER(CacheDesc), p]
+        L.pa_prefill_chunk.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, p, p, f32, p, p,
+                                       C.POINTER(CacheDesc), p]
         L.pa_get_last_device_error.argtypes = [C.POINTER(C.c_uint32), p]
         L.pa_decode_noalloc.argtypes = [p, p, p, p, p, p, i32, i32, i32, f32, p, p, i32, C.POINTER(CacheDesc), p]
         L.pa_status_string.argtypes = [C.c_int]
@@ -247,7 +248,7 @@ def prefill_chunk(out, q, cu_q_lens, prefix_lens, block_tables, k_cache, v_cache
     ks, vs = _scales(desc, k_scale, v_scale, dev)
     _check("pa_prefill_chunk", lib().pa_prefill_chunk(
         _ptr(out), _ptr(q), _ptr(cu_q_lens), _ptr(prefix_lens), _ptr(block_tables), n, block_tables.shape[1], Hq,
-        int(max_q_len), _ptr(k_cache), _ptr(v_cache), float(scale), _ptr(ks), _ptr(vs), C.byref(desc),
+        int(max_q_len), total, _ptr(k_cache), _ptr(v_cache), float(scale), _ptr(ks), _ptr(vs), C.byref(desc),
         _stream(stream)))
 
 

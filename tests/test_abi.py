@@ -88,11 +88,13 @@ def test_write_and_copy_reject_bad_arguments_on_host():
 
 def test_prefill_rejects_bad_arguments_on_host():
     L = ops.lib()
-    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 32, 64, FAKE, FAKE, 0.1, None, None,
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 32, 64, 100, FAKE, FAKE, 0.1, None, None,
                               C.byref(desc(dt=1)), None) == -2  # fp8 prefill not built
-    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 30, 64, FAKE, FAKE, 0.1, None, None,
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 30, 64, 100, FAKE, FAKE, 0.1, None, None,
                               C.byref(desc()), None) == -1
-    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 32, 64, FAKE, FAKE, 0.1, None, None,
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 128, 64, 100, FAKE, FAKE, 0.1, None, None,
+                              C.byref(desc()), None) == -2  # group of 16 not built
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 8, 32, 64, 100, FAKE, FAKE, 0.1, None, None,
                               C.byref(desc()), None) == 0
 
 
