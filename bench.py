@@ -47,6 +47,13 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured (cuBLAS bf16 GEMM, burst)"
+    return 1590.0, "fallback"
+
+
 def file_sha(path):
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
@@ -347,6 +354,103 @@ def run_ours(args, rank, world, device):
                 k_scale=k_scale, v_scale=v_scale, q=q, pool=pool)
 
 
+# ----------------------------------------------------- mixed decode + prefill
+class _StaticStep:
+    """Stand-in for a trace: one fixed step, repeated."""
+
+    def __init__(self, name, Hq, Hkv, D, seqs, pool):
+        from types import SimpleNamespace
+        self.name, self.Hq, self.Hkv, self.D, self.fp8 = name, Hq, Hkv, D, False
+        self.sched = SimpleNamespace(num_preemptions=0, cfg=SimpleNamespace(max_num_seqs=seqs),
+                                     alloc=SimpleNamespace(num_blocks=pool))
+
+
+def prefill_flops(cu_q, prefix_lens, Hq, D):
+    """Algorithmic FLOPs of causal chunked prefill: per chunk of C queries over
+    a prefix of P keys, C*P + C(C+1)/2 query-key pairs, 4*D flops per pair
+    (q.k and p.v), for every query head."""
+    C = np.diff(np.asarray(cu_q, np.int64))
+    P = np.asarray(prefix_lens, np.int64)
+    return int((Hq * 4 * D * (C * P + C * (C + 1) // 2)).sum())
+
+
+def run_mixed(args, rank, world, device):
+    """The mixed step: 192 decode sequences (lognormal lengths, median 1024,
+    capped at 8192) plus 8 prefill chunks of 512 tokens over prefixes uniform
+    in [0, 4096], 32/8 heads, head_dim 128, bf16.  One step = write every new
+    token's K/V, decode, prefill; the same step is repeated."""
+    import torch
+
+    from paged_kv_cache_408_b200 import inputs as I
+    from paged_kv_cache_408_b200 import ops
+
+    torch.cuda.set_device(device)
+    dc, pc = I.mixed_step(args.seed + rank)
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    def it(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a, dt)).to(device)
+
+    dk, dv = bf(dc.k_cache), bf(dc.v_cache)
+    pk, pv = bf(pc.k_cache), bf(pc.v_cache)
+    dq, pq = bf(dc.q), bf(pc.q)
+    dout, pout = torch.empty_like(dq), torch.empty_like(pq)
+    dnk, dnv, dsl = bf(dc.new_k), bf(dc.new_v), it(dc.slot_mapping, np.int64)
+    pnk, pnv, psl = bf(pc.new_k), bf(pc.new_v), it(pc.slot_mapping, np.int64)
+    dbt, dl = it(dc.block_tables, np.int32), it(dc.seq_lens, np.int32)
+    pcu, ppf, pbt = it(pc.cu_q, np.int32), it(pc.prefix_lens, np.int32), it(pc.block_tables, np.int32)
+    ws = ops.alloc_workspace(dc.B, dc.Hq, dc.D, dc.block_tables.shape[1], args.partition, device=device)
+    flush = L2Flush(torch, device)
+    st = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(st)
+        ops.write_kv(dnk, dnv, dsl, dk, dv)
+        ops.write_kv(pnk, pnv, psl, pk, pv)
+        if evs:
+            evs[1].record(st)
+        ops.decode(dout, dq, dk, dv, dbt, dl, dc.scale, workspace=ws, partition_tokens=args.partition)
+        if evs:
+            evs[2].record(st)
+        ops.prefill_chunk(pout, pq, pcu, ppf, pbt, pk, pv, pc.scale, pc.max_q_len)
+        if evs:
+            evs[3].record(st)
+        return 4
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    launches = 0
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda._sleep(int(2e7 + 1e6 * args.steps))
+        for e in ev:
+            flush()
+            launches += step(e)
+        torch.cuda.synchronize()
+    if ops.get_last_device_error():
+        raise RuntimeError("device status word set during the mixed step")
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    pre_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    kvb_step = kv_bytes(dc.seq_lens, dc.Hkv, dc.D, 2)
+    tr = _StaticStep("192 decode seqs (lognormal, median 1024) + 8 prefill chunks x 512 over U[0,4096] "
+                     "prefixes, 32/8 heads, d128, bf16", dc.Hq, dc.Hkv, dc.D, dc.B + len(pc.prefix_lens),
+                     dc.num_blocks + pc.k_cache.shape[0])
+    return dict(tot_ms=sum(step_ms), step_ms=step_ms, dec_ms=dec_ms, kvb=kvb_step * args.steps,
+                seqsteps=dc.B * args.steps, algb=[decode_alg_bytes(dc.seq_lens, dc.Hq, dc.Hkv, dc.D, 2)] * args.steps,
+                launches=launches, clocks=clk.summary(), e2e=None, plan_ms=0.0, tr=tr, plans=None, fp8=False,
+                prefill={"ms": sum(pre_ms) / len(pre_ms), "flops": prefill_flops(pc.cu_q, pc.prefix_lens, pc.Hq, pc.D),
+                         "tokens": int(pc.cu_q[-1])})
+
+
 # ------------------------------------------------------------ oracle timing
 def oracle_step_time(plan, kc, vc, q, Hq, scale, ks, vs, rows, nthreads):
     import oracle
@@ -477,7 +581,7 @@ def main():
         torch.cuda.set_device(device)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
-    r = run_ours(args, rank, world, device)
+    r = run_mixed(args, rank, world, device) if args.workload == "mixed" else run_ours(args, rank, world, device)
 
     tot_s = r["tot_ms"] / 1e3
     kvb, seqsteps = r["kvb"], r["seqsteps"]
@@ -517,7 +621,15 @@ def main():
             line["e2e"] = {"value": e["kvb"] / (e["ms"] / 1e3) / 1e9, "unit": "GB/s",
                            "h2d_bytes_per_step": int(e["h2d"]), "d2h_bytes_per_step": int(e["d2h"]),
                            "ms_per_step": e["ms"] / args.steps}
-        if world == 1 and not args.no_cpu_baseline:
+        if r.get("prefill"):
+            pf = r["prefill"]
+            tfl = pf["flops"] / (pf["ms"] / 1e3) / 1e12
+            bf16_peak, kind = tensor_peak()
+            line["prefill"] = {"tflops": tfl, "ms_per_launch": pf["ms"], "flops_per_launch": pf["flops"],
+                               "tokens": pf["tokens"],
+                               "roofline": {"bound": "tensor", "achieved": tfl, "peak": bf16_peak, "unit": "TFLOP/s",
+                                            "frac": tfl / bf16_peak, "peak_kind": kind, "kernel": "pa_prefill_chunk"}}
+        if world == 1 and not args.no_cpu_baseline and r.get("plans"):
             import torch as _t
             kc, vc = host_copy(r["k_cache"], _t), host_copy(r["v_cache"], _t)
             qh = host_copy(r["q"], _t)
