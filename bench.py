@@ -548,6 +548,22 @@ def workload_config(args, tr):
 
 
 # ---------------------------------------------------------------- driver
+def aggregate(tot_s, kv_bytes_done, seq_steps, world, device):
+    """Whole-job figures over independent replicas: the slowest rank's device
+    time and the work of all ranks (weak scaling: no data-path collective,
+    only this reduction of the measurements)."""
+    if world <= 1:
+        return tot_s, kv_bytes_done, seq_steps
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([tot_s], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    w = torch.tensor([kv_bytes_done, seq_steps], device=device, dtype=torch.float64)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(w[0].item()), float(w[1].item())
+
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -583,16 +599,7 @@ def main():
 
     r = run_mixed(args, rank, world, device) if args.workload == "mixed" else run_ours(args, rank, world, device)
 
-    tot_s = r["tot_ms"] / 1e3
-    kvb, seqsteps = r["kvb"], r["seqsteps"]
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([tot_s], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        w = torch.tensor([kvb, seqsteps], device=device, dtype=torch.float64)
-        dist.all_reduce(w, op=dist.ReduceOp.SUM)
-        tot_s = float(t.item())
-        kvb, seqsteps = float(w[0].item()), float(w[1].item())
+    tot_s, kvb, seqsteps = aggregate(r["tot_ms"] / 1e3, r["kvb"], r["seqsteps"], world, device)
 
     if rank == 0:
         peak, peak_kind = peaks()

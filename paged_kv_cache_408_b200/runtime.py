@@ -224,6 +224,9 @@ class Scheduler:
 
     # -- requests
     def add_request(self, seq: Sequence) -> None:
+        if blocks_for(seq.num_tokens) > self.cfg.max_blocks_per_seq:
+            raise ValueError(f"request {seq.seq_id}: {seq.num_tokens} tokens exceed the "
+                             f"{self.cfg.max_blocks_per_seq}-block table")
         seq.status = WAITING
         if seq.prefill_end == 0 and seq.fresh:
             seq.prefill_end = seq.num_tokens
@@ -330,8 +333,8 @@ class Scheduler:
                 budget -= got
         while budget > 0 and self.waiting and len(self.running) < self.cfg.max_num_seqs:
             s = self.waiting[0]
-            if not self._can_admit(s):
-                break
+            if s.seq_id in plan.preempted or not self._can_admit(s):
+                break  # a sequence evicted in this step waits at least one step
             self.waiting.popleft()
             self.add_running(s)
             plan.admitted.append(s.seq_id)
@@ -371,6 +374,7 @@ class Scheduler:
     def complete(self, plan: StepPlan) -> None:
         """Advance the sequences of the step the caller has just run."""
         decode, chunks = self._inflight
+        cap = BLOCK_SIZE * self.cfg.max_blocks_per_seq
         for s in decode:
             if s.status != RUNNING:
                 continue
@@ -378,6 +382,8 @@ class Scheduler:
             s.prefill_end = s.num_cached
             s.num_tokens = s.num_cached + 1
             s.decode_left -= 1
+            if s.num_cached >= cap:  # the block table is full: the sequence ends here
+                s.decode_left = 0
         for s, start, n in chunks:
             if s.status != RUNNING:
                 continue
