@@ -281,8 +281,8 @@ def run_ours(args, rank, world, device):
 
     # ---- timed: inputs resident in HBM, L2 flushed between steps (outside the events)
     timed = dsteps[args.warmup:]
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
     launches = 0
     if world > 1:
         import torch.distributed as dist
@@ -290,22 +290,31 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
         # hold the stream while the host enqueues every timed step, so the
-        # events see device time only (no host launch gaps)
+        # events see device time only (no host launch gaps).  Only the step
+        # is bracketed: an event between two kernels would cut the
+        # programmatic launch chain (write -> decode -> merge -> prefill).
         torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
-        for ds, (e0, e1, e2, e3) in zip(timed, ev):
+        for ds, (e0, e1) in zip(timed, ev):
             flush()
             e0.record(st)
             launches += launch(ds, q, out, new_k, new_v, pq, pout)
-            e1.record(st)
             launches += decode(ds, q, out)
-            e2.record(st)
             launches += prefill(ds, pq, pout)
-            e3.record(st)
+            e1.record(st)
+        torch.cuda.synchronize()
+        # the decode call alone (its kernel and the merge), same steps and
+        # cache, for the roofline of the dominant kernel
+        torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
+        for ds, (e0, e1) in zip(timed, dev_ev):
+            flush()
+            e0.record(st)
+            decode(ds, q, out)
+            e1.record(st)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms = [e0.elapsed_time(e3) for e0, _, _, e3 in ev]
-    dec_ms = [e1.elapsed_time(e2) for _, e1, e2, _ in ev]
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    dec_ms = [e0.elapsed_time(e1) for e0, e1 in dev_ev]
     tot_ms = sum(step_ms)
     kvb = sum(kv_bytes(ds.plan.decode_lens, Hkv, D, eb) for ds in timed)
     seqsteps = sum(ds.B for ds in timed)
@@ -405,41 +414,48 @@ def run_mixed(args, rank, world, device):
     flush = L2Flush(torch, device)
     st = torch.cuda.current_stream()
 
-    def step(evs=None):
-        if evs:
-            evs[0].record(st)
+    def write():
         ops.write_kv(dnk, dnv, dsl, dk, dv)
         ops.write_kv(pnk, pnv, psl, pk, pv)
-        if evs:
-            evs[1].record(st)
+
+    def decode():
         ops.decode(dout, dq, dk, dv, dbt, dl, dc.scale, workspace=ws, partition_tokens=args.partition)
-        if evs:
-            evs[2].record(st)
+
+    def prefill():
         ops.prefill_chunk(pout, pq, pcu, ppf, pbt, pk, pv, pc.scale, pc.max_q_len)
-        if evs:
-            evs[3].record(st)
-        return 4
+
+    def step():
+        write()
+        decode()
+        prefill()
+        return 5  # two writes, decode + merge, prefill
+
+    def timed(fn, n):
+        """n calls of fn, each bracketed by events, L2 flushed in between."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        torch.cuda._sleep(int(2e7 + 1e6 * n))
+        for e0, e1 in ev:
+            flush()
+            e0.record(st)
+            fn()
+            e1.record(st)
+        torch.cuda.synchronize()
+        return [e0.elapsed_time(e1) for e0, e1 in ev]
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    launches = 0
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda._sleep(int(2e7 + 1e6 * args.steps))
-        for e in ev:
-            flush()
-            launches += step(e)
-        torch.cuda.synchronize()
+        step_ms = timed(step, args.steps)  # the whole step: one programmatic launch chain
+        dec_ms = timed(decode, args.steps)  # then each kernel alone, for its roofline
+        pre_ms = timed(prefill, args.steps)
+    launches = 5 * args.steps
     if ops.get_last_device_error():
         raise RuntimeError("device status word set during the mixed step")
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    pre_ms = [e[2].elapsed_time(e[3]) for e in ev]
     kvb_step = kv_bytes(dc.seq_lens, dc.Hkv, dc.D, 2)
     tr = _StaticStep("192 decode seqs (lognormal, median 1024) + 8 prefill chunks x 512 over U[0,4096] "
                      "prefixes, 32/8 heads, d128, bf16", dc.Hq, dc.Hkv, dc.D, dc.B + len(pc.prefix_lens),
@@ -543,7 +559,7 @@ def run_reference(args, rank, world):
 def workload_config(args, tr):
     return {"workload": tr.name, "trace": args.workload, "seqs": tr.sched.cfg.max_num_seqs, "q_heads": tr.Hq,
             "kv_heads": tr.Hkv, "head_dim": tr.D, "block_size": 16, "cache_dtype": "fp8_e4m3" if tr.fp8 else "bf16",
-            "pool_blocks": tr.sched.alloc.num_blocks, "partition_tokens": args.partition or 256,
+            "pool_blocks": tr.sched.alloc.num_blocks, "partition_tokens": args.partition or "balanced",
             "l2": "flushed between steps outside the timed events (256 MiB written, then 256 MiB read)", "parallelism": "replicas"}
 
 

@@ -174,13 +174,12 @@ int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head
  *                       positions, so each sequence's result is bitwise
  *                       independent of the rest of the batch.
  *   workspace     device scratch of at least pa_decode_workspace_size()
- *                 bytes, 256-byte aligned.  It must be zero-filled before
- *                 its first use (e.g. cudaMemset); its first bytes hold the
- *                 per-(sequence, kv head) arrival counters of the in-kernel
- *                 split-K merge, which every completed call leaves at zero,
- *                 so later calls (any batch size) need no re-initialisation.
- *                 Calls that share one workspace must not overlap on the
- *                 GPU.
+ *                 bytes, 256-byte aligned: the split-K pieces (fp32
+ *                 outputs, log2-sum-exps and piece counts) that a second
+ *                 kernel, enqueued by the same call, merges.  Every call
+ *                 writes all it reads, so it needs no initialisation and
+ *                 keeps nothing between calls.  Calls that share one
+ *                 workspace must not overlap on the GPU.
  * num_seqs must be in [0, 2048] (0 enqueues nothing); num_kv_heads <= 128;
  * num_q_heads / num_kv_heads in {1,2,4,8}.
  */
@@ -238,10 +237,10 @@ int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const i
  *     (cudaGetSymbolAddress, once per device, with that device current);
  *     make that first call before any stream capture.
  *   - Every call on a device shares the one array and it keeps the last
- *     call's contents; each call first clears (cudaMemsetAsync on `stream`)
- *     the part that must start at zero.  Calls that overlap on the GPU (on
- *     different streams without ordering) race on the array and give wrong
- *     results: order them.
+ *     call's contents; a call writes every part it reads, so nothing is
+ *     cleared between calls.  Calls that overlap on the GPU (on different
+ *     streams without ordering) race on the array and give wrong results:
+ *     order them.
  */
 #define PA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
 

@@ -139,21 +139,15 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     rc = resolve_partition(partition_tokens, &P);
     if (rc != PA_OK) return rc;
     const int max_parts = pa::decode_max_parts(max_blocks_per_seq, P);
-    int *counters = nullptr;
-    float *ws_o = nullptr, *ws_lse = nullptr;
+    pa::DecodeArgs a{out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
+                     num_q_heads, desc->num_kv_heads, desc->head_dim, desc->num_blocks, scale, k_scale, v_scale,
+                     P, max_parts, nullptr, nullptr, nullptr, fp8, status_word_ptr()};
     if (max_parts > 1) {
         const size_t need = pa::decode_ws_bytes(num_seqs, num_q_heads, desc->head_dim, max_parts);
         if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
             return PA_ERR_WORKSPACE;
-        char *base = static_cast<char *>(workspace);
-        counters = reinterpret_cast<int *>(base);
-        ws_o = reinterpret_cast<float *>(base + pa::decode_ws_counter_bytes());
-        ws_lse = reinterpret_cast<float *>(base + pa::decode_ws_counter_bytes() +
-                                           pa::decode_ws_o_bytes(num_seqs, num_q_heads, desc->head_dim, max_parts));
+        pa::decode_ws_carve(workspace, num_seqs, num_q_heads, desc->head_dim, max_parts, a);
     }
-    pa::DecodeArgs a{out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
-                     num_q_heads, desc->num_kv_heads, desc->head_dim, desc->num_blocks, scale, k_scale, v_scale,
-                     P, max_parts, counters, ws_o, ws_lse, fp8, status_word_ptr()};
     return from_cuda(pa::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -64,6 +64,35 @@ PA_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 200
     return true;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Every libpa kernel is launched as a programmatic dependent of the kernel
+// before it on the stream (launch_pdl below).  Its CTAs may then be
+// scheduled while that kernel drains, which hides the launch latency;
+// pdl_wait(), placed before the kernel's first global memory access, returns
+// once the preceding grid has completed with all its memory operations
+// visible, so the ordering is that of a plain launch whatever that kernel
+// is.  pdl_trigger() lets the next kernel be scheduled.  Both are no-ops
+// when there is no programmatic dependency.
+PA_DEVICE void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+PA_DEVICE void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // ------------------------------------------------------- 1-D bulk async copy
 // Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned) completing on `bar` as a transaction.  No multicast.

@@ -1,5 +1,5 @@
 // decode.cu -- paged decode attention for sm_100a, with split-K pieces and
-// an in-kernel log-sum-exp merge.
+// a log-sum-exp merge kernel launched as a programmatic dependent.
 //
 // What is computed ("Production Serving: Continuous Batching and
 // PagedAttention", The Build, Step 6 "Implement attention over paged
@@ -16,20 +16,28 @@
 //    warp's per-item latencies (q load, epilogue, merge) are hidden by the
 //    other warps of the SM.
 //  * Work split (host selects with partition_tokens):
-//      balanced -- the (sequence, kv head, block) triples of the batch form
-//        one line; warp g takes the contiguous share [g*S, (g+1)*S) with
-//        S = ceil(total / warps): every warp streams the same number of
-//        bytes whatever the length mix;
+//      balanced -- the (sequence, kv head) segments of the batch form one
+//        line in cost units: one unit per 16-token block plus kSegmentCost
+//        units charged at the head of every segment for its per-item work
+//        (q load, epilogue, output write); warp g takes the contiguous share
+//        [g*S, (g+1)*S) with S = ceil(total / warps), so warps get the same
+//        time's work whatever the length mix;
 //      fixed -- every (sequence, kv head) is cut into partitions of P tokens,
 //        dealt round-robin to warps (full partitions first); split points
 //        depend only on token positions, so results are batch-invariant.
 //    Every CTA rebuilds the split from seq_lens with a block-wide scan in
 //    shared memory: no host sync, no empty CTAs for short sequences.
+//  * One CTA of 12 warps per SM.  With several CTAs per SM the warp
+//    schedulers favour the CTA that arrived first, so equal shares finished
+//    up to 15% apart; warps of one CTA are served evenly.  (GQA groups of 8
+//    keep two CTAs of 4 warps: their arithmetic per byte is twice as high
+//    and there the uneven service measured faster.)
 //  * Each warp runs its own NSTAGE-deep shared-memory ring filled by 1-D
 //    bulk async copies (the TMA engine; K and V of one block of one kv head
-//    are 4 KB contiguous each) that complete on mbarriers.  The producer
-//    runs ahead across item boundaries and keeps block-table entries in
-//    registers (a sliding window, plus the next item's first entries).
+//    are 4 KB contiguous each) that complete on mbarriers.  The rings of an
+//    SM's warps fill kRingBytes of shared memory.  The producer runs ahead
+//    across item boundaries and keeps block-table entries in registers (a
+//    sliding window, plus the next item's first entries).
 //  * Math on CUDA cores (4-8 query rows per step are far below a
 //    tensor-core tile): lanes form token groups of LPT lanes; a lane owns
 //    DPL head dims (16-byte shared-memory reads, bank-conflict-free), keeps
@@ -42,9 +50,12 @@
 //    the sum taken against the same max, so the result is the exact softmax.
 //  * A (sequence, kv head) covered by one piece is written as bf16 straight
 //    from registers.  Otherwise each piece writes its fp32 output and its
-//    log2-sum-exp to the workspace and bumps an arrival counter; the warp
-//    that completes the last piece merges all pieces by log-sum-exp and
-//    resets the counter (the workspace stays ready for the next call).
+//    log2-sum-exp to the workspace with plain stores: no fence and no
+//    atomic on the streaming warps (a gpu-scope fence waits for the store
+//    acknowledgements, microseconds while HBM is saturated).  A second
+//    kernel, launched as a programmatic dependent so that its launch
+//    overlaps the decode kernel, merges the pieces by log-sum-exp once the
+//    decode grid has completed.
 #include <algorithm>
 #include <mutex>
 
@@ -56,6 +67,8 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 256 before a rescale
+constexpr int kSegmentCost = 2;            // balanced split: cost units charged per segment
+constexpr size_t kRingBytes = 192 * 1024;  // K/V staging rings of all warps of an SM
 constexpr unsigned kFull = 0xffffffffu;
 
 PA_DEVICE float lg2(float x) {
@@ -83,11 +96,16 @@ struct Cfg {
     static constexpr int NS = TSUB * G;               // partial scores per lane per sub-step
     static constexpr bool RS = NS >= LPT;             // reduce-scatter (else all-reduce)
     static constexpr int VPL = RS ? NS / LPT : NS;    // scores a lane owns after the reduction
-    static constexpr int NW = 4;                      // warps per CTA
+    // CTAS CTAs of NW warps per SM share the register file (G = 8 needs ~255
+    // registers a thread, so 8 warps an SM; otherwise ~168, so 12) and a
+    // kRingBytes shared-memory ring, split into NSTAGE stages per warp.
+    static constexpr int CTAS = (G >= 8) ? 2 : 1;     // CTAs per SM
+    static constexpr int NW = (G >= 8) ? 4 : 12;      // warps per CTA
     static constexpr int NT = NW * 32;
-    static constexpr int NSTAGE = (G >= 8) ? 3 : 2;   // ring depth per warp
-    static constexpr int MIN_CTAS = (G >= 8) ? 2 : 3; // resident CTAs per SM the register budget targets
+    static constexpr int NSTAGE = (int)(kRingBytes / ((size_t)CTAS * NW * 2 * BLKB));  // ring depth per warp
+    static constexpr int MIN_CTAS = CTAS;
     static constexpr size_t STAGE_BYTES = (size_t)NW * NSTAGE * 2 * BLKB;
+    static_assert(NSTAGE >= 2 && NSTAGE <= 32, "ring depth");
     static_assert(LPT >= 1 && LPT <= 32 && 32 % LPT == 0, "bad lane split");
     static_assert(TPG * NGRP == 16 && TSUB * NSUB == TPG, "bad token split");
     static_assert(!RS || NS % LPT == 0, "reduce-scatter needs NS divisible by LPT");
@@ -238,20 +256,24 @@ struct Schedule {
         return it;
     }
 
-    // balanced: the piece that starts at line position pos, cut at `end`
-    PA_DEVICE Item balanced_item(int pos, int end) const {
-        Item it;
+    // balanced: the piece of the segment holding line position pos, cut at
+    // `end`.  A segment is kSegmentCost cost units, then one unit per block;
+    // its pieces are the warp shares that hold its block units.  Returns the
+    // line position after the piece (nblk <= 0: the share ends before the
+    // segment's first block).
+    PA_DEVICE int balanced_item(int pos, int end, Item &it) const {
         it.b = upper_index(pre0, B, pos);
         it.len = len[it.b];
-        const int nb = (it.len + 15) >> 4;
+        const int nb = (it.len + 15) >> 4, U = nb + kSegmentCost;
         const int u = pos - pre0[it.b];
-        it.kvh = u / nb;
-        it.blk0 = u - it.kvh * nb;
-        const int seg0 = pre0[it.b] + it.kvh * nb, seg1 = seg0 + nb;
-        it.nblk = min(seg1, end) - pos;
-        it.piece = pos / S - seg0 / S;
-        it.npieces = (seg1 - 1) / S - seg0 / S + 1;
-        return it;
+        it.kvh = u / U;
+        const int seg0 = pre0[it.b] + it.kvh * U, r0 = seg0 + kSegmentCost, seg1 = seg0 + U;
+        const int p = max(pos, r0), stop = min(seg1, end);
+        it.blk0 = p - r0;
+        it.nblk = stop - p;
+        it.piece = p / S - r0 / S;
+        it.npieces = (seg1 - 1) / S - r0 / S + 1;
+        return stop;
     }
 };
 
@@ -271,14 +293,16 @@ struct ItemIter {
         }
     }
     PA_DEVICE bool next(const Schedule &sc, Item &it) {
-        if (cur >= end) return false;
         if (sc.P == 0) {
-            it = sc.balanced_item(cur, end);
-            cur += it.nblk;
-        } else {
-            it = sc.fixed_item(cur);
-            cur += step;
+            while (cur < end) {
+                cur = sc.balanced_item(cur, end, it);
+                if (it.nblk > 0) return true;
+            }
+            return false;
         }
+        if (cur >= end) return false;
+        it = sc.fixed_item(cur);
+        cur += step;
         return true;
     }
 };
@@ -380,78 +404,6 @@ PA_DEVICE void load_row(const uint8_t *row, const int (&choff)[C::NCH], float2 (
     }
 }
 
-// Log-sum-exp merge of the npieces partial results of one (sequence, kv
-// head) by a single warp: out = sum_p w_p o_p / sum_p w_p with
-// w_p = 2^(lse_p - max lse).  Pieces are read in chunks of CH with every load
-// of a chunk in flight at once (one L2 round trip per chunk, all heads
-// together); the running max is moved between chunks.
-template <class C>
-PA_DEVICE void merge_pieces(const DecodeArgs &a, size_t row0, int np, int lane) {
-    constexpr int D = C::D, E = D / 32, G = C::G, CH = 2;
-    float M[G], L[G], acc[G][E];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        M[h] = -INFINITY;
-        L[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
-    }
-    for (int p0 = 0; p0 < np; p0 += CH) {
-        float lp[G][CH], ov[G][CH][E];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float *lse = a.ws_lse + (row0 + h) * a.max_parts;
-            const float *op = a.ws_o + (row0 + h) * a.max_parts * D + lane * E;
-#pragma unroll
-            for (int u = 0; u < CH; ++u) {
-                const int p = p0 + u;
-                lp[h][u] = (p < np) ? __ldcg(lse + p) : -INFINITY;
-                if constexpr (E == 4) {
-                    const float4 v = (p < np) ? __ldcg(reinterpret_cast<const float4 *>(op + (size_t)p * D))
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
-                    ov[h][u][0] = v.x;
-                    ov[h][u][1] = v.y;
-                    ov[h][u][2] = v.z;
-                    ov[h][u][3] = v.w;
-                } else {
-                    const float2 v = (p < np) ? __ldcg(reinterpret_cast<const float2 *>(op + (size_t)p * D))
-                                              : make_float2(0.f, 0.f);
-                    ov[h][u][0] = v.x;
-                    ov[h][u][1] = v.y;
-                }
-            }
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float mx = M[h];
-#pragma unroll
-            for (int u = 0; u < CH; ++u) mx = fmaxf(mx, lp[h][u]);
-            if (mx == -INFINITY) continue;
-            const float sc = (M[h] == -INFINITY) ? 0.f : ex2(M[h] - mx);
-            M[h] = mx;
-            L[h] *= sc;
-#pragma unroll
-            for (int e = 0; e < E; ++e) acc[h][e] *= sc;
-#pragma unroll
-            for (int u = 0; u < CH; ++u) {
-                const float wgt = (lp[h][u] == -INFINITY) ? 0.f : ex2(lp[h][u] - mx);
-                L[h] += wgt;
-#pragma unroll
-                for (int e = 0; e < E; ++e) acc[h][e] += wgt * ov[h][u][e];
-            }
-        }
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-        const float inv = (L[h] > 0.f) ? 1.f / L[h] : 0.f;
-        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (row0 + h) * D + lane * E;
-#pragma unroll
-        for (int e = 0; e < E; e += 2)
-            *reinterpret_cast<__nv_bfloat162 *>(out + e) =
-                __floats2bfloat162_rn(acc[h][e] * inv, acc[h][e + 1] * inv);
-    }
-}
-
 // Raw inputs of one item that the consumer loads ahead of time: its q rows
 // (this lane's chunks, head slot h = head h ^ sh) and the fp8 scales.
 template <class C>
@@ -488,10 +440,12 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     const int g = lane / LPT, sub = lane % LPT;
     const int B = a.B, Hkv = a.Hkv, P = a.partition_tokens;  // P == 0: balanced split
     const int gw = blockIdx.x * NW + w, GW = gridDim.x * NW;
+    pdl_trigger();  // the merge kernel may be scheduled now; it waits for this grid
+    pdl_wait();     // the preceding kernel (e.g. the K/V write) has completed
 
     // ---- lengths, then exclusive scans over sequences: the balanced split
-    // needs each sequence's offset in the line (Hkv * blocks), the fixed one
-    // the numbers of full partitions and of ragged tails.
+    // needs each sequence's offset in the line (Hkv segments of cost units),
+    // the fixed one the numbers of full partitions and of ragged tails.
     const int cap = a.max_blocks * 16;
     for (int b = tid; b < B; b += C::NT) {
         int len = a.seq_lens[b];
@@ -505,7 +459,9 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     fence_mbar_init();
     __syncthreads();
     {
-        auto count0 = [&](int len) { return P == 0 ? Hkv * ((len + 15) >> 4) : len / P; };
+        auto count0 = [&](int len) {
+            return P == 0 ? (len > 0 ? Hkv * (((len + 15) >> 4) + kSegmentCost) : 0) : len / P;
+        };
         auto count1 = [&](int len) { return P == 0 ? 0 : (int)((len % P) != 0); };
         const int per = (B + C::NT - 1) / C::NT;  // each thread scans a run of sequences
         const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
@@ -739,9 +695,10 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
                     }
                 }
             }
+            if (lane == 0 && a.ws_np) a.ws_np[(size_t)it.b * Hkv + it.kvh] = 1;  // nothing to merge
         } else {
-            // ---- split-K: write this piece, count it; the warp completing
-            // the last piece of this (sequence, kv head) merges them all
+            // ---- split-K: this piece's normalised output and log2-sum-exp;
+            // piece 0 also records how many pieces the merge kernel combines
             if (g == 0) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
@@ -758,25 +715,102 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
                     if (sub == 0)  // sub 0 has sh == 0: slot h is head h
                         a.ws_lse[(row0 + h) * a.max_parts + it.piece] = (l[h] > 0.f) ? m[h] + lg2(l[h]) : -INFINITY;
                 }
-                __threadfence();
             }
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) {
-                int *ctr = a.counters + (size_t)it.b * Hkv + it.kvh;
-                last = atomicAdd(ctr, 1) == it.npieces - 1;
-                if (last) *ctr = 0;  // every piece has arrived: ready for the next call
-            }
-            last = __shfl_sync(kFull, last, 0);
-            if (last) {
-                __threadfence();
-                merge_pieces<C>(a, row0, it.npieces, lane);
-            }
+            if (lane == 0 && it.piece == 0) a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces;
         }
         it = nx;
         have = have_nx;
         have_nx = have && items.next(sc, nx);
     }
+}
+
+// Log-sum-exp merge of the split-K pieces, one warp per (sequence, q head):
+//     out = sum_p w_p o_p / sum_p w_p,   w_p = 2^(lse_p - max_p lse_p)
+// where o_p is piece p's normalised output and lse_p its log2-sum-exp.  Runs
+// as a programmatic dependent of the decode kernel: its CTAs may become
+// resident while the decode grid drains, and griddepcontrol.wait returns
+// once that grid has completed with its memory visible.  Lane l owns head
+// dims [l*E, l*E + E).  The length, the piece count and the first kFirst
+// pieces are loaded together (addresses do not depend on the count; slots
+// past it are in bounds and ignored), so up to kFirst pieces cost one L2
+// round trip.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
+    constexpr int E = D / 32, kFirst = 8;
+    pdl_trigger();
+    pdl_wait();
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);  // b * Hq + h
+    if (row >= (long long)a.B * a.Hq) return;
+    const int b = (int)(row / a.Hq), h = (int)(row % a.Hq), kvh = h / (a.Hq / a.Hkv);
+    const float *lse = a.ws_lse + (size_t)row * a.max_parts;
+    const float *op = a.ws_o + (size_t)row * a.max_parts * D + lane * E;
+    auto load_o = [&](int p, float (&v)[E]) {
+        if constexpr (E == 4) {
+            const float4 x = __ldcg(reinterpret_cast<const float4 *>(op + (size_t)p * D));
+            v[0] = x.x;
+            v[1] = x.y;
+            v[2] = x.z;
+            v[3] = x.w;
+        } else {
+            const float2 x = __ldcg(reinterpret_cast<const float2 *>(op + (size_t)p * D));
+            v[0] = x.x;
+            v[1] = x.y;
+        }
+    };
+    const int len = __ldcg(a.seq_lens + b);
+    const int np = __ldcg(a.ws_np + (size_t)b * a.Hkv + kvh);
+    float lp[kFirst], v[kFirst][E];
+#pragma unroll
+    for (int u = 0; u < kFirst; ++u)
+        if (u < a.max_parts) {
+            lp[u] = __ldcg(lse + u);
+            load_o(u, v[u]);
+        }
+    if (len <= 0 || len > a.max_blocks * 16) return;  // empty or rejected: the decode kernel wrote the row
+    if (np <= 1) return;                               // one piece: the decode kernel wrote the row
+    if (np > a.max_parts) {
+        if (lane == 0) flag_error(a.err, PA_DEVERR_BAD_LEN);
+        return;
+    }
+    // chunks of kFirst pieces, each chunk's loads in flight together; the
+    // running max moves between chunks
+    float M = -INFINITY, L = 0.f, acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int p0 = 0; p0 < np; p0 += kFirst) {
+        if (p0 > 0) {
+#pragma unroll
+            for (int u = 0; u < kFirst; ++u)
+                if (p0 + u < np) {
+                    lp[u] = __ldcg(lse + p0 + u);
+                    load_o(p0 + u, v[u]);
+                }
+        }
+        float mc = M;
+#pragma unroll
+        for (int u = 0; u < kFirst; ++u)
+            if (p0 + u < np) mc = fmaxf(mc, lp[u]);  // slots past np may hold anything: never read
+        if (mc == -INFINITY) continue;
+        const float sc = (M == -INFINITY) ? 0.f : ex2(M - mc);
+        M = mc;
+        L *= sc;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] *= sc;
+#pragma unroll
+        for (int u = 0; u < kFirst; ++u)
+            if (p0 + u < np && lp[u] != -INFINITY) {
+                const float w = ex2(lp[u] - M);
+                L += w;
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] = fmaf(w, v[u][e], acc[e]);
+            }
+    }
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + (size_t)row * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+        *reinterpret_cast<__nv_bfloat162 *>(out + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
 }
 
 template <class C>
@@ -824,8 +858,10 @@ cudaError_t run(const DecodeArgs &a, cudaStream_t st) {
                                 ? (long long)a.Hkv * a.B * a.max_blocks / kMinShareBlocks + 1
                                 : (long long)a.Hkv * a.B * a.max_parts;
     const long long grid = std::max<long long>(1, std::min<long long>((units + C::NW - 1) / C::NW, ctas));
-    decode_kernel<C><<<(unsigned)grid, C::NT, smem, st>>>(a);
-    return cudaGetLastError();
+    e = launch_pdl(decode_kernel<C>, dim3((unsigned)grid), dim3(C::NT), smem, st, a);
+    if (e != cudaSuccess || !a.ws_np) return e;  // no workspace: every (sequence, kv head) is one piece
+    const long long rows = (long long)a.B * a.Hq;
+    return launch_pdl(merge_kernel<C::D>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st, a);
 }
 
 template <int D, bool FP8>
@@ -841,16 +877,23 @@ cudaError_t by_group(const DecodeArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-size_t decode_ws_counter_bytes() { return (size_t)kMaxDecodeSeqs * kMaxDecodeKvHeads * sizeof(int); }
-
-size_t decode_ws_o_bytes(int B, int Hq, int D, int max_parts) {
-    const size_t o = (size_t)B * Hq * max_parts * D * sizeof(float);
-    return (o + 255) & ~(size_t)255;
+namespace {
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+size_t ws_np_bytes(int B, int Hq) { return round256((size_t)B * Hq * sizeof(int)); }  // >= B * Hkv
+size_t ws_o_bytes(int B, int Hq, int D, int max_parts) {
+    return round256((size_t)B * Hq * max_parts * D * sizeof(float));
 }
+}  // namespace
 
 size_t decode_ws_bytes(int B, int Hq, int D, int max_parts) {
-    const size_t lse = (size_t)B * Hq * max_parts * sizeof(float);
-    return decode_ws_counter_bytes() + decode_ws_o_bytes(B, Hq, D, max_parts) + ((lse + 255) & ~(size_t)255);
+    return ws_np_bytes(B, Hq) + ws_o_bytes(B, Hq, D, max_parts) + round256((size_t)B * Hq * max_parts * sizeof(float));
+}
+
+void decode_ws_carve(void *base, int B, int Hq, int D, int max_parts, DecodeArgs &a) {
+    char *p = static_cast<char *>(base);
+    a.ws_np = reinterpret_cast<int *>(p);
+    a.ws_o = reinterpret_cast<float *>(p + ws_np_bytes(B, Hq));
+    a.ws_lse = reinterpret_cast<float *>(p + ws_np_bytes(B, Hq) + ws_o_bytes(B, Hq, D, max_parts));
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {

@@ -7,8 +7,8 @@
 #include "common.cuh"
 #include "kernels.h"
 
-// The scratch: arrival counters, partial outputs and partial log-sum-exps of
-// the in-kernel split-K merge.  Every GPU that loads the library holds it
+// The scratch: piece counts, partial outputs and partial log-sum-exps of the
+// split-K merge.  Every GPU that loads the library holds it
 // until the process exits.  Host code must not use this name as an address
 // (on the host it is only a stand-in); it uses the address looked up below.
 static __device__ __align__(256) unsigned char pa_noalloc_scratch[PA_DECODE_NOALLOC_SCRATCH_BYTES];
@@ -68,25 +68,16 @@ extern "C" int pa_decode_noalloc(void *out, const void *q, const void *k_cache, 
     const size_t need = max_parts > 1 ? pa::decode_ws_bytes(num_seqs, num_q_heads, desc->head_dim, max_parts) : 0;
     if (need > PA_DECODE_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
 
-    int *counters = nullptr;
-    float *ws_o = nullptr, *ws_lse = nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pa::DecodeArgs a{out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
+                     num_q_heads, desc->num_kv_heads, desc->head_dim, desc->num_blocks, scale, k_scale, v_scale,
+                     P, max_parts, nullptr, nullptr, nullptr, fp8, pa::status_word()};
     if (max_parts > 1) {
         void *scratch = nullptr;
         const int rc = scratch_address(&scratch);
         if (rc != PA_OK) return rc;
-        char *base = static_cast<char *>(scratch);
-        counters = reinterpret_cast<int *>(base);
-        ws_o = reinterpret_cast<float *>(base + pa::decode_ws_counter_bytes());
-        ws_lse = reinterpret_cast<float *>(base + pa::decode_ws_counter_bytes() +
-                                           pa::decode_ws_o_bytes(num_seqs, num_q_heads, desc->head_dim, max_parts));
-        // the arrival counters of this call's (sequence, kv head) pairs must start at zero
-        const size_t nctr = (size_t)num_seqs * desc->num_kv_heads * sizeof(int);
-        if (cudaMemsetAsync(counters, 0, nctr, st) != cudaSuccess) return PA_ERR_CUDA;
+        pa::decode_ws_carve(scratch, num_seqs, num_q_heads, desc->head_dim, max_parts, a);
     }
-    pa::DecodeArgs a{out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
-                     num_q_heads, desc->num_kv_heads, desc->head_dim, desc->num_blocks, scale, k_scale, v_scale,
-                     P, max_parts, counters, ws_o, ws_lse, fp8, pa::status_word()};
     const cudaError_t e = pa::launch_decode(a, st);
     if (e == cudaSuccess) return PA_OK;
     return e == cudaErrorNotSupported ? PA_ERR_UNSUPPORTED : PA_ERR_CUDA;

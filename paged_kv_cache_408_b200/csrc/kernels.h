@@ -41,7 +41,7 @@ struct DecodeArgs {
     const float *k_scale, *v_scale;
     int partition_tokens;  // 0: balanced split; else a multiple of 16 (fixed partitions)
     int max_parts;         // most pieces one (sequence, kv head) can be cut into
-    int *counters;         // [kMaxDecodeSeqs * kMaxDecodeKvHeads] arrivals per (seq, kv head); zero between calls
+    int *ws_np;            // [B][Hkv] pieces of each (sequence, kv head), written by every call
     float *ws_o;           // [B][Hq][max_parts][D]
     float *ws_lse;         // [B][Hq][max_parts]
     bool fp8;
@@ -68,21 +68,21 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
 // Device address of the status word on the current device (nullptr if unknown).
 unsigned *status_word();
 
-// Workspace layout shared by pa_decode_workspace_size and pa_decode:
-// [arrival counters | partial outputs | partial log2-sum-exp].  The counter
-// region has a fixed size so it never overlaps data of a call with another
-// batch size; it must be zero before the first call and every call leaves it
-// zero.
+// Workspace layout shared by pa_decode_workspace_size, pa_decode and
+// pa_decode_noalloc: [piece counts | partial outputs | partial log2-sum-exp],
+// each region 256-byte aligned.  Every call writes what it reads (the decode
+// kernel writes the piece counts and partials, the merge kernel reads them),
+// so the workspace needs no initialisation and keeps nothing between calls.
 constexpr int kMaxDecodeSeqs = 2048;
-constexpr int kMinShareBlocks = 16;  // balanced split: smallest per-CTA share, in blocks
+constexpr int kMinShareBlocks = 16;  // balanced split: smallest per-warp share, in cost units
 constexpr int kMaxDecodeKvHeads = 128;
-size_t decode_ws_counter_bytes();
 // Pieces one (sequence, kv head) of max_blocks blocks can be cut into.
 inline int decode_max_parts(int max_blocks, int partition_tokens) {
     return partition_tokens == 0 ? max_blocks / kMinShareBlocks + 2
                                  : (max_blocks * 16 + partition_tokens - 1) / partition_tokens;
 }
-size_t decode_ws_o_bytes(int B, int Hq, int D, int max_parts);
 size_t decode_ws_bytes(int B, int Hq, int D, int max_parts);
+// Points a.ws_np / a.ws_o / a.ws_lse into a workspace of decode_ws_bytes().
+void decode_ws_carve(void *base, int B, int Hq, int D, int max_parts, DecodeArgs &a);
 
 }  // namespace pa

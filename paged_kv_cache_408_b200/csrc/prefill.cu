@@ -82,6 +82,8 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int c = blockIdx.z, kvh = blockIdx.y;
     const int i0 = blockIdx.x * C::QPOS;
+    pdl_trigger();
+    pdl_wait();
     const int q_start = a.cu_q[c];
     const int clen = a.cu_q[c + 1] - q_start;
     const int pfx = a.prefix_lens[c];
@@ -356,8 +358,7 @@ cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
     const int64_t rows = a.num_blocks * a.Hkv * 16;
     if (!cache_map(&tk, a.k_cache, rows, C::D) || !cache_map(&tv, a.v_cache, rows, C::D)) return cudaErrorInvalidValue;
     dim3 grid((a.max_q_len + C::QPOS - 1) / C::QPOS, a.Hkv, a.n_chunks);
-    prefill_kernel<C><<<grid, C::NT, C::SMEM, st>>>(a, tk, tv);
-    return cudaGetLastError();
+    return launch_pdl(prefill_kernel<C>, grid, dim3(C::NT), C::SMEM, st, a, tk, tv);
 }
 
 template <int D>

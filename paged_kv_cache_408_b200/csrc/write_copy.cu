@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4 *__restrict__
                                                        int Hkv, int D, int64_t num_blocks, void *__restrict__ kc,
                                                        void *__restrict__ vc, const float *__restrict__ ks,
                                                        const float *__restrict__ vs, unsigned *err) {
+    pdl_trigger();
+    pdl_wait();
     const int cpr = D / 8;  // chunks per (token, head) row
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_chunks;
          i += (int64_t)gridDim.x * blockDim.x) {
@@ -80,6 +82,8 @@ __global__ void __launch_bounds__(256) write_kv_kernel(const uint4 *__restrict__
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4 *__restrict__ kc, uint4 *__restrict__ vc,
                                                           const int32_t *__restrict__ pairs, int64_t num_blocks,
                                                           int64_t vecs, unsigned *err) {
+    pdl_trigger();
+    pdl_wait();
     const int64_t s = pairs[2 * blockIdx.x], d = pairs[2 * blockIdx.x + 1];
     if (s < 0 || d < 0 || s >= num_blocks || d >= num_blocks) {
         if (threadIdx.x == 0) flag_error(err, PA_DEVERR_BAD_PAIR);
@@ -97,24 +101,17 @@ cudaError_t launch_write_kv(const WriteArgs &a, cudaStream_t st) {
     const int threads = 256;
     int64_t blocks = (n_chunks + threads - 1) / threads;
     if (blocks > 148 * 64) blocks = 148 * 64;
-    if (a.fp8)
-        write_kv_kernel<true><<<(unsigned)blocks, threads, 0, st>>>(
-            (const uint4 *)a.k, (const uint4 *)a.v, a.slots, n_chunks, a.Hkv, a.D, a.num_blocks, a.k_cache,
-            a.v_cache, a.k_scale, a.v_scale, a.err);
-    else
-        write_kv_kernel<false><<<(unsigned)blocks, threads, 0, st>>>(
-            (const uint4 *)a.k, (const uint4 *)a.v, a.slots, n_chunks, a.Hkv, a.D, a.num_blocks, a.k_cache,
-            a.v_cache, a.k_scale, a.v_scale, a.err);
-    return cudaGetLastError();
+    return launch_pdl(a.fp8 ? write_kv_kernel<true> : write_kv_kernel<false>, dim3((unsigned)blocks), dim3(threads),
+                      0, st, (const uint4 *)a.k, (const uint4 *)a.v, a.slots, n_chunks, a.Hkv, a.D, a.num_blocks,
+                      a.k_cache, a.v_cache, a.k_scale, a.v_scale, a.err);
 }
 
 cudaError_t launch_copy_blocks(const CopyArgs &a, cudaStream_t st) {
     if (a.num_pairs == 0) return cudaSuccess;
     const int64_t vecs = (int64_t)a.Hkv * 16 * a.D * a.elem_bytes / 16;
     dim3 grid((unsigned)a.num_pairs, 2);
-    copy_blocks_kernel<<<grid, 256, 0, st>>>((uint4 *)a.k_cache, (uint4 *)a.v_cache, a.pairs, a.num_blocks, vecs,
-                                             a.err);
-    return cudaGetLastError();
+    return launch_pdl(copy_blocks_kernel, grid, dim3(256), 0, st, (uint4 *)a.k_cache, (uint4 *)a.v_cache, a.pairs,
+                      a.num_blocks, vecs, a.err);
 }
 
 }  // namespace pa

@@ -171,8 +171,8 @@ def decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, p
 
 
 def alloc_workspace(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, partition_tokens=0, device=None):
-    """Caller-side helper: a zero-filled torch buffer large enough for
-    pa_decode (the library needs it zeroed once; calls keep it that way)."""
+    """Caller-side helper: a torch buffer large enough for pa_decode (it
+    needs no particular contents; zero-filled here only to be deterministic)."""
     n = decode_workspace_size(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, partition_tokens)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
