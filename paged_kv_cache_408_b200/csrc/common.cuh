@@ -123,6 +123,21 @@ PA_DEVICE float2 fmul2(float2 a, float2 b) {
     return d;
 }
 
+PA_DEVICE float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(reinterpret_cast<unsigned long long &>(d))
+        : "l"(reinterpret_cast<unsigned long long &>(a)), "l"(reinterpret_cast<unsigned long long &>(b)));
+    return d;
+}
+
+// Three-input maximum (sm_100).
+PA_DEVICE float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 2^x with the hardware approximation (MUFU.EX2), flushing denormal results.
 PA_DEVICE float ex2(float x) {
     float y;

@@ -9,25 +9,37 @@
 // the block table -- the prefix already in the cache and the chunk's own
 // keys, written there first.
 //
-// Design:
-//  * One CTA (4 warps) per (chunk, kv head, tile of 128/G query positions).
-//    Its 128 accumulator rows are those positions x the G query heads of
-//    the kv head (row = position*G + head), so every K/V tile is fetched
-//    once per GQA group.
-//  * K and V are streamed in tiles of 128 keys = 8 paged blocks.  Each
-//    block of one kv head is a 16-row x D slab of the cache; warp 0 gathers
-//    the 8 slabs through the block table with 2-D TMA tensor copies
-//    (64-column boxes, 128-byte swizzle, no multicast) straight into the
-//    operand layout of the tensor cores.  K and V buffers are double
-//    buffered with their own mbarriers.
-//  * S = Q K^T (M=128, N=128 keys, K=D) and O += P V (M=128, N=D, K=128
-//    keys) are tcgen05.mma kind::f16 (bf16 in, fp32 accumulate) issued by
-//    one thread; S and O live in TMEM.  Softmax reads S from TMEM (one
-//    thread per row), applies the causal mask, moves the running max only
-//    when it grows by more than 8 (log2 units) -- then it rescales its O
-//    row in TMEM -- and writes P as bf16 to shared memory for the second
-//    MMA.  The P.V MMA of tile j-1 overlaps S and softmax of tile j.
-//  * Key rows past the sequence end in the last tile are zeroed in shared
+// Design (warp-specialised, two query tiles per CTA):
+//  * A query tile is 128 accumulator rows = 128/G positions x the G query
+//    heads of one kv head (row = position*G + head), so every K/V tile is
+//    fetched once per GQA group.  A CTA holds two query tiles of the same
+//    (chunk, kv head) that share every K/V tile.
+//  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of query
+//    tiles 0 and 1 (thread = accumulator row = TMEM lane); warp 8 gathers
+//    K/V tiles of 128 keys (8 paged blocks) through the block table with
+//    2-D TMA tensor copies (64-column boxes, 128-byte swizzle, no multicast)
+//    into a ring of K and V slots; one lane of warp 9 issues the tcgen05
+//    MMAs (kind::f16, bf16 in, fp32 accumulate) and commits them to
+//    mbarriers.
+//  * Per K/V tile j and query tile t: S_t = Q_t K_j^T into TMEM; softmax
+//    warpgroup t reads S_t, writes P_t as bf16 into the first half of the
+//    same TMEM columns, and O_t += P_t V_j reads P_t straight from TMEM (the
+//    A operand of the MMA), so P never goes through shared memory and the
+//    tensor core's shared-memory reads are only Q, K and V.  The two query
+//    tiles alternate: the tensor core works on one tile's products while
+//    the other tile's softmax runs.
+//  * S_t(j+1) is issued only after O_t += P_t(j) V_j has completed (it
+//    overwrites P_t), so when softmax t sees S_t(j+1) the previous P.V is
+//    done and a rescale of its O row in TMEM is safe.
+//  * Softmax applies the causal mask only on tiles that reach past the
+//    row's position, moves the running max only when it grows by more than
+//    8 (log2 units), and computes P with one packed FMA and one MUFU.EX2
+//    per score.
+//  * Every mbarrier is waited on in phase order and never falls two phases
+//    behind its producer (a parity wait cannot tell phase k from k+2); the
+//    protocol was checked against that rule, and for deadlock, by a
+//    discrete simulation over random schedules.
+//  * Key rows past the sequence end in the last V tile are zeroed in shared
 //    memory before P.V, so stale cache contents can never reach the output.
 #include <cudaTypedefs.h>
 
@@ -46,76 +58,100 @@ constexpr float kRescaleThreshold = 8.0f;
 template <int D_, int G_>
 struct PCfg {
     static constexpr int D = D_, G = G_;
-    static constexpr int M = 128;                 // accumulator rows per CTA
-    static constexpr int QPOS = M / G;            // query positions per CTA
-    static constexpr int KT = 128;                // keys per K/V tile
+    static constexpr int M = 128;                 // accumulator rows of a query tile
+    static constexpr int QPOS = M / G;            // query positions per query tile
+    static constexpr int NQ = 2;                  // query tiles per CTA
+    static constexpr int KT = 128;                // keys per K/V tile (8 blocks)
     static constexpr int NATOM = D / 64;          // 128-byte column atoms along D
-    static constexpr int ATOM = 128 * 128;        // bytes of one atom column of a 128-row tile
-    static constexpr int TILE = NATOM * ATOM;     // bytes of a Q, K or V tile
+    static constexpr int QATOM = M * 128;         // bytes of one atom column of a query tile
+    static constexpr int KATOM = KT * 128;        // bytes of one atom column of a K/V tile
+    static constexpr int QTILE = NATOM * QATOM;
+    static constexpr int KTILE = NATOM * KATOM;
+    static constexpr int NSLOT = (D == 128) ? 2 : 4;  // K and V ring depth
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = TILE;            // two K tiles
-    static constexpr int OFF_V = 3 * TILE;        // two V tiles
-    static constexpr int OFF_P = 5 * TILE;        // P: 128 rows x 128 keys (two atoms)
-    static constexpr int OFF_BAR = OFF_P + 2 * ATOM;
-    static constexpr int SMEM = OFF_BAR + 128 + 1024;  // barriers + alignment slack
-    static constexpr int NT = 128;
-    static constexpr uint32_t TMEM_COLS = 256;
-    static constexpr uint32_t COL_S = 0, COL_O = 128;
-    static constexpr uint32_t TX_BYTES = 8 * NATOM * 16 * 128;  // one K or V tile
+    static constexpr int OFF_K = OFF_Q + NQ * QTILE;
+    static constexpr int OFF_V = OFF_K + NSLOT * KTILE;
+    static constexpr int OFF_BAR = OFF_V + NSLOT * KTILE;
+    static constexpr int NBAR = 4 * NSLOT + 4 * NQ + 1;  // K/V full+empty; S full, P full, O done, O final; end
+    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // barriers, TMEM slot, alignment slack
+    static constexpr int NSMW = NQ * 4;           // softmax warps
+    static constexpr int W_LOAD = NSMW, W_MMA = NSMW + 1;
+    static constexpr int NT = (NSMW + 2) * 32;
+    // TMEM columns: S_t (and P_t in its first KT/2 columns) at t * KT; O_t at COL_O + t * D
+    static constexpr uint32_t COL_O = NQ * KT;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t TX_BYTES = KTILE;   // one K or V tile
     static_assert(M % G == 0, "group must divide 128");
+    static_assert(COL_O + NQ * D <= TMEM_COLS, "TMEM columns");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
-    constexpr int D = C::D, G = C::G;
+    constexpr int D = C::D, G = C::G, KT = C::KT, NS = C::NSLOT, NQ = C::NQ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *sQ = smem + C::OFF_Q;
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
-    uint8_t *sP = smem + C::OFF_P;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *barK = bars, *barV = bars + 2, *barS = bars + 4, *barO = bars + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    uint64_t *kfull = bars, *kempty = bars + NS, *vfull = bars + 2 * NS, *vempty = bars + 3 * NS;
+    uint64_t *sfull = bars + 4 * NS, *pfull = sfull + NQ, *odone = pfull + NQ, *ofinal = odone + NQ;
+    uint64_t *mma_done = ofinal + NQ;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int c = blockIdx.z, kvh = blockIdx.y;
-    const int i0 = blockIdx.x * C::QPOS;
+    const int i0 = blockIdx.x * (NQ * C::QPOS);
     pdl_trigger();
     pdl_wait();
     const int q_start = a.cu_q[c];
     const int clen = a.cu_q[c + 1] - q_start;
     const int pfx = a.prefix_lens[c];
-    if (i0 >= clen) return;  // this tile lies past the chunk (uniform per CTA)
+    if (i0 >= clen) return;  // this CTA's positions lie past the chunk (uniform per CTA)
     const int L = pfx + clen;
     if (clen < 0 || pfx < 0 || L > a.max_blocks * 16 || q_start < 0 || q_start + clen > a.total_q) {
         if (tid == 0) flag_error(a.err, PA_DEVERR_BAD_LEN);
         return;
     }
-    const int nvalid = min(C::QPOS, clen - i0);
-    const int n_keys = pfx + i0 + nvalid;  // keys the last valid row sees
-    const int ntiles = (n_keys + C::KT - 1) / C::KT;
-    const int nalloc = (L + 15) >> 4;     // blocks of the sequence
+    const int nalloc = (L + 15) >> 4;  // blocks of the sequence
     const int32_t *bt = a.block_tables + (size_t)c * a.max_blocks;
-
-    if (w == 0) tmem_alloc(tmem_slot, C::TMEM_COLS);
-    if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
-        fence_mbar_init();
+    // K/V tiles each query tile needs (causal: up to its last valid row)
+    int ntl[NQ], ntiles = 0;
+#pragma unroll
+    for (int t = 0; t < NQ; ++t) {
+        const int first = i0 + t * C::QPOS;
+        const int nv = max(0, min(C::QPOS, clen - first));
+        ntl[t] = nv > 0 ? (pfx + first + nv + KT - 1) / KT : 0;
+        ntiles = max(ntiles, ntl[t]);
     }
 
-    // ---- Q tile: row t = (position t / G, head t % G), 128-byte swizzle
-    const int my_i = tid / G, my_h = tid % G;
-    const bool row_valid = my_i < nvalid;
-    {
-        const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
-                                   ((size_t)(q_start + i0 + my_i) * a.Hq + (size_t)kvh * G + my_h) * D;
+    if (w == C::W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    if (tid == 0) {
+        for (int i = 0; i < 4 * NS; ++i) mbar_init(&bars[i], 1);
+        for (int t = 0; t < NQ; ++t) {
+            mbar_init(&sfull[t], 1);
+            mbar_init(&pfull[t], 128);
+            mbar_init(&odone[t], 1);
+            mbar_init(&ofinal[t], 1);
+        }
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+    }
+    // ---- query tiles: row r of tile t = (position r / G, head r % G), 128-byte swizzle
+    if (w < C::NSMW) {
+        const int t = w / 4, r = tid & 127;
+        const int ip = i0 + t * C::QPOS + r / G;
+        const bool valid = ip < clen;
+        const __nv_bfloat16 *src =
+            static_cast<const __nv_bfloat16 *>(a.q) + ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D;
+        uint8_t *dst = sQ + t * C::QTILE + r * 128;
 #pragma unroll
         for (int ch = 0; ch < D / 8; ++ch) {
-            const uint4 v = row_valid ? *reinterpret_cast<const uint4 *>(src + ch * 8) : make_uint4(0, 0, 0, 0);
+            const uint4 v = valid ? *reinterpret_cast<const uint4 *>(src + ch * 8) : make_uint4(0, 0, 0, 0);
             const int at = ch / 8, cc = ch % 8;
-            *reinterpret_cast<uint4 *>(sQ + at * C::ATOM + tid * 128 + ((cc ^ (tid & 7)) * 16)) = v;
+            *reinterpret_cast<uint4 *>(dst + at * C::QATOM + ((cc ^ (r & 7)) * 16)) = v;
         }
     }
     fence_proxy_async_smem();
@@ -123,188 +159,218 @@ __global__ void __launch_bounds__(C::NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    bool ok = true;
 
-    // ---- warp 0 gathers the 8 blocks of a K or V tile through the block table
-    auto issue = [&](int j, bool is_v) {
-        uint64_t *bar = is_v ? &barV[j & 1] : &barK[j & 1];
-        uint8_t *dst = (is_v ? sV : sK) + (j & 1) * C::TILE;
-        const CUtensorMap *map = is_v ? &tmV : &tmK;
-        if (lane == 0) mbar_arrive_expect_tx(bar, C::TX_BYTES);
-        __syncwarp();
-        if (lane < 8) {
-            const int lb = min(j * 8 + lane, nalloc - 1);  // past the end: a valid block, masked later
-            int phys = bt[lb];
-            if (phys < 0 || phys >= a.num_blocks) {
+    if (w == C::W_LOAD) {
+        // ---- producer: K tile j, then V tile j, into ring slot j % NS.  The
+        // warp keeps a window of 32 block-table entries in registers (lane l
+        // holds entry win0 + l), refilled every 32/BPT tiles, so a tile's
+        // copies are issued without a global round trip.
+        constexpr int BPT = KT / 16;  // blocks per tile
+        int win0 = 0, went = bt[min(lane, nalloc - 1)];
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % NS;
+            const uint32_t use = j / NS;  // how many times slot s was filled before
+            if (j * BPT + BPT > win0 + 32) {
+                win0 = j * BPT;
+                went = bt[min(win0 + lane, nalloc - 1)];
+            }
+            // lanes 0..BPT-1: block j*BPT + lane (past the end: the last block, masked later)
+            int phys = __shfl_sync(0xffffffffu, went, (min(j * BPT + lane % BPT, nalloc - 1) - win0) & 31);
+            if (lane < BPT && (phys < 0 || phys >= a.num_blocks)) {
                 flag_error(a.err, PA_DEVERR_BAD_BLOCK);
                 phys = 0;
             }
             const int row = (phys * a.Hkv + kvh) * 16;
 #pragma unroll
-            for (int at = 0; at < C::NATOM; ++at) tma_load_2d(dst + at * C::ATOM + lane * 16 * 128, map, at * 64, row, bar);
-        }
-    };
-    if (w == 0) {
-        issue(0, false);
-        issue(0, true);
-        if (ntiles > 1) {
-            issue(1, false);
-            issue(1, true);
-        }
-    }
-
-    const int pos = pfx + i0 + my_i;
-    const float sl2 = a.scale * kLog2e;
-    const uint32_t lane_base = tmem + ((uint32_t)(w * 32) << 16);
-    constexpr uint32_t idS = idesc_bf16_f32(128, C::KT, false);
-    constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
-    float m = -INFINITY, l = 0.f;
-    bool dead = false;
-
-    for (int j = 0; j < ntiles && !dead; ++j) {
-        const int b = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        // ---- S = Q K^T
-        bool ok = mbar_wait(&barK[b], ph);
-        if (tid == 0 && ok) {
-            tc_fence_after();
-            const uint32_t q0 = smem_addr(sQ), k0 = smem_addr(sK + b * C::TILE);
+            for (int kv = 0; kv < 2; ++kv) {
+                uint64_t *full = kv ? &vfull[s] : &kfull[s];
+                if (use > 0) ok = mbar_wait(kv ? &vempty[s] : &kempty[s], (use - 1) & 1) && ok;
+                if (lane == 0) mbar_arrive_expect_tx(full, C::TX_BYTES);
+                __syncwarp();
+                if (lane < BPT) {
+                    uint8_t *dst = (kv ? sV : sK) + s * C::KTILE + lane * 16 * 128;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk / 4) * C::ATOM + (kk % 4) * 32;
-                tc_mma_bf16(tmem + C::COL_S, smem_desc_sw128(q0 + off, 16, 1024), smem_desc_sw128(k0 + off, 16, 1024),
-                            idS, kk > 0);
+                    for (int at = 0; at < C::NATOM; ++at)
+                        tma_load_2d(dst + at * C::KATOM, kv ? &tmV : &tmK, at * 64, row, full);
+                }
+                __syncwarp();
             }
-            tc_commit(barS);
         }
-        ok = mbar_wait(barS, j & 1) && ok;
-        tc_fence_after();
-        if (w == 0 && j + 2 < ntiles) issue(j + 2, false);  // K buffer b is free again
-
-        // ---- softmax of this thread's row
-        float s[C::KT];
+    } else if (w == C::W_MMA) {
+        // ---- MMA issue, per K/V tile j: S_t(j) for both query tiles, then
+        // O_t += P_t(j) V_j as each softmax warpgroup hands over P_t(j)
+        constexpr uint32_t idS = idesc_bf16_f32(128, KT, false);
+        constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % NS;
+            ok = mbar_wait(&kfull[s], (j / NS) & 1) && ok;
 #pragma unroll
-        for (int q = 0; q < C::KT / 32; ++q) {
-            float t32[32];
-            tmem_ld32(lane_base + C::COL_S + 32 * q, t32);
+            for (int t = 0; t < NQ; ++t) {
+                if (j < ntl[t]) {
+                    // P_t(j-1), in S_t's columns, has been consumed
+                    if (j > 0) ok = mbar_wait(&odone[t], (j - 1) & 1) && ok;
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t q0 = smem_addr(sQ + t * C::QTILE), k0 = smem_addr(sK + s * C::KTILE);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) s[32 * q + e] = t32[e];
-        }
-        tmem_wait_ld();
-        const int kv0 = j * C::KT;
-        float mt = -INFINITY;
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            tc_mma_bf16(tmem + t * KT, smem_desc_sw128(q0 + (kk / 4) * C::QATOM + (kk % 4) * 32, 16, 1024),
+                                        smem_desc_sw128(k0 + (kk / 4) * C::KATOM + (kk % 4) * 32, 16, 1024), idS,
+                                        kk > 0);
+                        tc_commit(&sfull[t]);
+                    }
+                    __syncwarp();
+                }
+            }
+            if (lane == 0) tc_commit(&kempty[s]);
+            __syncwarp();
+            ok = mbar_wait(&vfull[s], (j / NS) & 1) && ok;
+            const int kv0 = j * KT;
+            if (kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
+                uint8_t *vt = sV + s * C::KTILE;
+                for (int r = max(L - kv0, 0) + lane; r < KT; r += 32)
 #pragma unroll
-        for (int e = 0; e < C::KT; ++e) {
-            s[e] = (row_valid && kv0 + e <= pos) ? s[e] * sl2 : -INFINITY;
-            mt = fmaxf(mt, s[e]);
-        }
-        const bool rescale = mt > m + kRescaleThreshold;
-        float alpha = 1.f;
-        if (rescale) {
-            alpha = (m == -INFINITY) ? 0.f : ex2(m - mt);
-            m = mt;
-            l *= alpha;
-        }
-        uint32_t pk[C::KT / 2];
-        float sum = 0.f;
+                    for (int at = 0; at < C::NATOM; ++at)
 #pragma unroll
-        for (int e = 0; e < C::KT; e += 2) {
-            const float p0 = (s[e] == -INFINITY) ? 0.f : ex2(s[e] - m);
-            const float p1 = (s[e + 1] == -INFINITY) ? 0.f : ex2(s[e + 1] - m);
-            sum += p0 + p1;
-            const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-            pk[e / 2] = *reinterpret_cast<const uint32_t *>(&bb);
+                        for (int cc = 0; cc < 8; ++cc)
+                            *reinterpret_cast<uint4 *>(vt + at * C::KATOM + r * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+#pragma unroll
+            for (int t = 0; t < NQ; ++t) {
+                if (j < ntl[t]) {
+                    ok = mbar_wait(&pfull[t], j & 1) && ok;  // P_t(j) is in TMEM
+                    if (lane == 0) {
+                        tc_fence_after();
+                        const uint32_t v0 = smem_addr(sV + s * C::KTILE);
+#pragma unroll
+                        for (int kk = 0; kk < KT / 16; ++kk)
+                            tc_mma_bf16_tmem_a(tmem + C::COL_O + t * D, tmem + t * KT + kk * 8,
+                                               smem_desc_sw128(v0 + kk * 16 * 128, C::KATOM, 1024), idO,
+                                               j > 0 || kk > 0);
+                        tc_commit(&odone[t]);
+                        if (j == ntl[t] - 1) tc_commit(&ofinal[t]);
+                    }
+                    __syncwarp();
+                }
+            }
+            if (lane == 0) tc_commit(&vempty[s]);
+            __syncwarp();
         }
-        l += sum;
-
-        // ---- P.V of the previous tile must be done before P and O are touched
-        if (j > 0) {
-            ok = mbar_wait(barO, (j - 1) & 1) && ok;
+        // every MMA of this CTA has completed before TMEM is released
+        if (lane == 0) tc_commit(mma_done);
+        __syncwarp();
+        ok = mbar_wait(mma_done, 0) && ok;
+    } else {
+        // ---- softmax of query tile t, one accumulator row per thread
+        const int t = w / 4, r = tid & 127;
+        const int ip = i0 + t * C::QPOS + r / G;
+        const bool row_valid = ip < clen;
+        const int pos = pfx + ip;
+        const float sl2 = a.scale * kLog2e;
+        const uint32_t lane_base = tmem + ((uint32_t)((w & 3) * 32) << 16);
+        float m = -INFINITY, l = 0.f;
+        for (int j = 0; j < ntl[t]; ++j) {
+            ok = mbar_wait(&sfull[t], j & 1) && ok;
             tc_fence_after();
-            if (w == 0 && j + 1 < ntiles) issue(j + 1, true);  // its V buffer is free again
+            float sv[KT];
+#pragma unroll
+            for (int q = 0; q < KT / 32; ++q) {
+                float t32[32];
+                tmem_ld32(lane_base + t * KT + 32 * q, t32);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) sv[32 * q + e] = t32[e];
+            }
+            tmem_wait_ld();
+            // raw scores (the scale is positive, so the max commutes with it);
+            // the causal mask only where the tile reaches past this row
+            const int kv0 = j * KT;
+            if (!(row_valid && kv0 + KT - 1 <= pos)) {
+#pragma unroll
+                for (int e = 0; e < KT; ++e) sv[e] = (row_valid && kv0 + e <= pos) ? sv[e] : -INFINITY;
+            }
+            float mraw = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < KT; e += 2) mraw = fmax3(mraw, sv[e], sv[e + 1]);
+            const float mt = mraw * sl2;
+            const bool rescale = mt > m + kRescaleThreshold;
+            float alpha = 1.f;
+            if (rescale) {
+                alpha = (m == -INFINITY) ? 0.f : ex2(m - mt);
+                m = mt;
+                l *= alpha;
+            }
+            // p = 2^(s*scale*log2e - m): one packed FMA and one MUFU.EX2 per
+            // score; masked scores are -inf and give 2^-inf = 0
+            const float mb = (m == -INFINITY) ? 0.f : m;
+            const float2 sc2 = make_float2(sl2, sl2), nb2 = make_float2(-mb, -mb);
+            float2 sum2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int h = 0; h < KT / 64; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const float2 x = ffma2(make_float2(sv[64 * h + e], sv[64 * h + e + 1]), sc2, nb2);
+                    const float p0 = ex2(x.x), p1 = ex2(x.y);
+                    sum2 = fadd2(sum2, make_float2(p0, p1));
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+                    pk[e / 2] = *reinterpret_cast<const uint32_t *>(&bb);
+                }
+                tmem_st32_u(lane_base + t * KT + 32 * h, pk);  // P over the S columns just read
+            }
+            l += sum2.x + sum2.y;
+            // O_t holds P.V up to tile j-1, complete (S_t(j) was issued after it):
+            // rescale in TMEM; tcgen05.ld/st are warp-collective, so the warp
+            // rescales if any of its rows needs it
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    float o[32];
+                    tmem_ld32(lane_base + C::COL_O + t * D + 32 * q, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                    tmem_st32(lane_base + C::COL_O + t * D + 32 * q, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&pfull[t]);
         }
-        // tcgen05.ld/st are warp-collective: rescale if any row of the warp needs it
-        // (rows that do not keep alpha == 1)
-        if (__any_sync(0xffffffffu, rescale) && j > 0) {
+        if (ntl[t] > 0) {
+            // ---- epilogue: O / l, bf16, one row per thread
+            ok = mbar_wait(&ofinal[t], 0) && ok;
+            tc_fence_after();
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
+                                 ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D;
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 float o[32];
-                tmem_ld32(lane_base + C::COL_O + 32 * q, o);
+                tmem_ld32(lane_base + C::COL_O + t * D + 32 * q, o);
                 tmem_wait_ld();
+                if (row_valid) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                tmem_st32(lane_base + C::COL_O + 32 * q, o);
-            }
-            tmem_wait_st();
-        }
+                    for (int e = 0; e < 32; e += 8) {
+                        uint32_t wds[4];
 #pragma unroll
-        for (int ch = 0; ch < C::KT / 8; ++ch) {
-            const int at = ch / 8, cc = ch % 8;
-            *reinterpret_cast<uint4 *>(sP + at * C::ATOM + tid * 128 + ((cc ^ (tid & 7)) * 16)) =
-                make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-        }
-        // ---- V tile: zero key rows past the sequence end (stale cache slots)
-        ok = mbar_wait(&barV[b], ph) && ok;
-        if (kv0 + tid >= L) {
-            uint8_t *vrow = sV + b * C::TILE + tid * 128;
-#pragma unroll
-            for (int at = 0; at < C::NATOM; ++at)
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    *reinterpret_cast<uint4 *>(vrow + at * C::ATOM + cc * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        dead = __syncthreads_or(!ok) != 0;
-        if (dead) break;
-        // ---- O += P V
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t p0 = smem_addr(sP), v0 = smem_addr(sV + b * C::TILE);
-#pragma unroll
-            for (int kk = 0; kk < C::KT / 16; ++kk) {
-                const uint32_t aoff = (kk / 4) * C::ATOM + (kk % 4) * 32;
-                tc_mma_bf16(tmem + C::COL_O, smem_desc_sw128(p0 + aoff, 16, 1024),
-                            smem_desc_sw128(v0 + kk * 16 * 128, C::ATOM, 1024), idO, j > 0 || kk > 0);
-            }
-            tc_commit(barO);
-        }
-    }
-
-    if (!dead) {
-        // ---- epilogue: O / l, bf16, one row per thread
-        const bool ok = mbar_wait(barO, (ntiles - 1) & 1);
-        tc_fence_after();
-        if (!ok && tid == 0) flag_error(a.err, PA_DEVERR_TIMEOUT);
-        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
-                             ((size_t)(q_start + i0 + my_i) * a.Hq + (size_t)kvh * G + my_h) * D;
-        const float inv = (l > 0.f) ? 1.f / l : 0.f;
-#pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-            float o[32];
-            tmem_ld32(lane_base + C::COL_O + 32 * q, o);
-            tmem_wait_ld();
-            if (row_valid) {
-#pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                    uint32_t wds[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const __nv_bfloat162 bb = __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
-                        wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
+                        for (int u = 0; u < 4; ++u) {
+                            const __nv_bfloat162 bb =
+                                __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
+                            wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
+                        }
+                        *reinterpret_cast<uint4 *>(dst + 32 * q + e) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
                     }
-                    *reinterpret_cast<uint4 *>(dst + 32 * q + e) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
                 }
             }
         }
-    } else if (tid == 0) {
-        flag_error(a.err, PA_DEVERR_TIMEOUT);
-        // let MMAs already issued finish before their TMEM is released
-        mbar_wait(barO, 0, 100000000ull);
-        mbar_wait(barO, 1, 100000000ull);
     }
+    if (!ok) flag_error(a.err, PA_DEVERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
-    if (w == 0) {
+    if (w == C::W_MMA) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -357,7 +423,7 @@ cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
     CUtensorMap tk, tv;
     const int64_t rows = a.num_blocks * a.Hkv * 16;
     if (!cache_map(&tk, a.k_cache, rows, C::D) || !cache_map(&tv, a.v_cache, rows, C::D)) return cudaErrorInvalidValue;
-    dim3 grid((a.max_q_len + C::QPOS - 1) / C::QPOS, a.Hkv, a.n_chunks);
+    dim3 grid((a.max_q_len + C::NQ * C::QPOS - 1) / (C::NQ * C::QPOS), a.Hkv, a.n_chunks);
     return launch_pdl(prefill_kernel<C>, grid, dim3(C::NT), C::SMEM, st, a, tk, tv);
 }
 
