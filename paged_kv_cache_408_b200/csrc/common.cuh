@@ -104,6 +104,11 @@ PA_DEVICE void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, ui
         : "memory");
 }
 
+// Named barrier `id` (1..15) over `nthreads` threads (a multiple of 32).
+PA_DEVICE void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ----------------------------------------------------------------- arithmetic
 // Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, lane-wise, RN.
 PA_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {

@@ -14,11 +14,12 @@
 //    heads of one kv head (row = position*G + head), so every K/V tile is
 //    fetched once per GQA group.  A CTA holds two query tiles of the same
 //    (chunk, kv head) that share every K/V tile.
-//  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of query
-//    tiles 0 and 1 (thread = accumulator row = TMEM lane); warp 8 gathers
+//  * Warp roles: warps 0-7 and 8-15 are the softmax warpgroups of query
+//    tiles 0 and 1 (two threads per accumulator row = TMEM lane, each with
+//    half of the row's keys and of its O columns); warp 16 gathers
 //    K/V tiles of 128 keys (8 paged blocks) through the block table with
 //    2-D TMA tensor copies (64-column boxes, 128-byte swizzle, no multicast)
-//    into a ring of K and V slots; one lane of warp 9 issues the tcgen05
+//    into a ring of K and V slots; one lane of warp 17 issues the tcgen05
 //    MMAs (kind::f16, bf16 in, fp32 accumulate) and commits them to
 //    mbarriers.
 //  * Per K/V tile j and query tile t: S_t = Q_t K_j^T into TMEM; softmax
@@ -71,10 +72,14 @@ struct PCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + NQ * QTILE;
     static constexpr int OFF_V = OFF_K + NSLOT * KTILE;
-    static constexpr int OFF_BAR = OFF_V + NSLOT * KTILE;
+    static constexpr int NSPLIT = 2;              // softmax threads per accumulator row
+    static constexpr int SCOL = KT / NSPLIT;      // S columns (keys) per softmax thread
+    static constexpr int OCOL = D / NSPLIT;       // O columns per softmax thread
+    static constexpr int OFF_X = OFF_V + NSLOT * KTILE;  // row max / sum exchange of a row's threads
+    static constexpr int OFF_BAR = OFF_X + 3 * NQ * NSPLIT * 128 * 4;
     static constexpr int NBAR = 4 * NSLOT + 4 * NQ + 1;  // K/V full+empty; S full, P full, O done, O final; end
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // barriers, TMEM slot, alignment slack
-    static constexpr int NSMW = NQ * 4;           // softmax warps
+    static constexpr int NSMW = NQ * 4 * NSPLIT;  // softmax warps
     static constexpr int W_LOAD = NSMW, W_MMA = NSMW + 1;
     static constexpr int NT = (NSMW + 2) * 32;
     // TMEM columns: S_t (and P_t in its first KT/2 columns) at t * KT; O_t at COL_O + t * D
@@ -84,6 +89,7 @@ struct PCfg {
     static_assert(M % G == 0, "group must divide 128");
     static_assert(COL_O + NQ * D <= TMEM_COLS, "TMEM columns");
     static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(SCOL % 64 == 0 && OCOL % 32 == 0, "whole TMEM column groups per thread");
 };
 
 template <class C>
@@ -100,6 +106,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     uint64_t *sfull = bars + 4 * NS, *pfull = sfull + NQ, *odone = pfull + NQ, *ofinal = odone + NQ;
     uint64_t *mma_done = ofinal + NQ;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+    float *xch = reinterpret_cast<float *>(smem + C::OFF_X);  // [3][NQ][NSPLIT][128]: max (2 parities), sum
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int c = blockIdx.z, kvh = blockIdx.y;
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         for (int i = 0; i < 4 * NS; ++i) mbar_init(&bars[i], 1);
         for (int t = 0; t < NQ; ++t) {
             mbar_init(&sfull[t], 1);
-            mbar_init(&pfull[t], 128);
+            mbar_init(&pfull[t], 128 * C::NSPLIT);
             mbar_init(&odone[t], 1);
             mbar_init(&ofinal[t], 1);
         }
@@ -141,14 +148,14 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
     // ---- query tiles: row r of tile t = (position r / G, head r % G), 128-byte swizzle
     if (w < C::NSMW) {
-        const int t = w / 4, r = tid & 127;
+        const int t = w / (4 * C::NSPLIT), half = (w / 4) % C::NSPLIT, r = (w % 4) * 32 + lane;
         const int ip = i0 + t * C::QPOS + r / G;
         const bool valid = ip < clen;
         const __nv_bfloat16 *src =
             static_cast<const __nv_bfloat16 *>(a.q) + ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D;
         uint8_t *dst = sQ + t * C::QTILE + r * 128;
 #pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch) {
+        for (int ch = half; ch < D / 8; ch += C::NSPLIT) {
             const uint4 v = valid ? *reinterpret_cast<const uint4 *>(src + ch * 8) : make_uint4(0, 0, 0, 0);
             const int at = ch / 8, cc = ch % 8;
             *reinterpret_cast<uint4 *>(dst + at * C::QATOM + ((cc ^ (r & 7)) * 16)) = v;
@@ -264,36 +271,49 @@ __global__ void __launch_bounds__(C::NT, 1)
         __syncwarp();
         ok = mbar_wait(mma_done, 0) && ok;
     } else {
-        // ---- softmax of query tile t, one accumulator row per thread
-        const int t = w / 4, r = tid & 127;
+        // ---- softmax of query tile t: NSPLIT threads per accumulator row,
+        // each with SCOL of the row's keys and OCOL of its O columns
+        constexpr int NSP = C::NSPLIT, SCOL = C::SCOL, OCOL = C::OCOL;
+        const int t = w / (4 * NSP), half = (w / 4) % NSP, r = (w % 4) * 32 + lane;
+        const int bar_id = 1 + t * 4 + (w % 4);  // named barrier of the NSP warps sharing these rows
         const int ip = i0 + t * C::QPOS + r / G;
         const bool row_valid = ip < clen;
         const int pos = pfx + ip;
         const float sl2 = a.scale * kLog2e;
         const uint32_t lane_base = tmem + ((uint32_t)((w & 3) * 32) << 16);
+        const uint32_t scol = t * KT + half * SCOL;            // this thread's S columns
+        const uint32_t pcol = t * KT + half * (SCOL / 2);      // its P words (two bf16 each)
+        const uint32_t ocol = C::COL_O + t * D + half * OCOL;  // its O columns
+        auto xslot = [&](int k, int hh) { return xch + ((k * NQ + t) * NSP + hh) * 128 + r; };
         float m = -INFINITY, l = 0.f;
         for (int j = 0; j < ntl[t]; ++j) {
             ok = mbar_wait(&sfull[t], j & 1) && ok;
             tc_fence_after();
-            float sv[KT];
+            float sv[SCOL];
 #pragma unroll
-            for (int q = 0; q < KT / 32; ++q) {
+            for (int q = 0; q < SCOL / 32; ++q) {
                 float t32[32];
-                tmem_ld32(lane_base + t * KT + 32 * q, t32);
+                tmem_ld32(lane_base + scol + 32 * q, t32);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) sv[32 * q + e] = t32[e];
             }
             tmem_wait_ld();
             // raw scores (the scale is positive, so the max commutes with it);
             // the causal mask only where the tile reaches past this row
-            const int kv0 = j * KT;
-            if (!(row_valid && kv0 + KT - 1 <= pos)) {
+            const int kv0 = j * KT + half * SCOL;
+            if (!(row_valid && kv0 + SCOL - 1 <= pos)) {
 #pragma unroll
-                for (int e = 0; e < KT; ++e) sv[e] = (row_valid && kv0 + e <= pos) ? sv[e] : -INFINITY;
+                for (int e = 0; e < SCOL; ++e) sv[e] = (row_valid && kv0 + e <= pos) ? sv[e] : -INFINITY;
             }
             float mraw = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < KT; e += 2) mraw = fmax3(mraw, sv[e], sv[e + 1]);
+            for (int e = 0; e < SCOL; e += 2) mraw = fmax3(mraw, sv[e], sv[e + 1]);
+            // the row's max over its threads; after this barrier every thread
+            // of the row has read its S columns, so P may overwrite them
+            *xslot(j & 1, half) = mraw;
+            named_bar_sync(bar_id, 32 * NSP);
+#pragma unroll
+            for (int hh = 0; hh < NSP; ++hh) mraw = fmaxf(mraw, *xslot(j & 1, hh));
             const float mt = mraw * sl2;
             const bool rescale = mt > m + kRescaleThreshold;
             float alpha = 1.f;
@@ -308,7 +328,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             const float2 sc2 = make_float2(sl2, sl2), nb2 = make_float2(-mb, -mb);
             float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int h = 0; h < KT / 64; ++h) {
+            for (int h = 0; h < SCOL / 64; ++h) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int e = 0; e < 64; e += 2) {
@@ -318,21 +338,21 @@ __global__ void __launch_bounds__(C::NT, 1)
                     const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
                     pk[e / 2] = *reinterpret_cast<const uint32_t *>(&bb);
                 }
-                tmem_st32_u(lane_base + t * KT + 32 * h, pk);  // P over the S columns just read
+                tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
             }
-            l += sum2.x + sum2.y;
+            l += sum2.x + sum2.y;  // this thread's keys; the row sum is combined at the end
             // O_t holds P.V up to tile j-1, complete (S_t(j) was issued after it):
             // rescale in TMEM; tcgen05.ld/st are warp-collective, so the warp
             // rescales if any of its rows needs it
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
+                for (int q = 0; q < OCOL / 32; ++q) {
                     float o[32];
-                    tmem_ld32(lane_base + C::COL_O + t * D + 32 * q, o);
+                    tmem_ld32(lane_base + ocol + 32 * q, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                    tmem_st32(lane_base + C::COL_O + t * D + 32 * q, o);
+                    tmem_st32(lane_base + ocol + 32 * q, o);
                 }
             }
             tmem_wait_st();
@@ -340,16 +360,21 @@ __global__ void __launch_bounds__(C::NT, 1)
             mbar_arrive(&pfull[t]);
         }
         if (ntl[t] > 0) {
-            // ---- epilogue: O / l, bf16, one row per thread
+            // ---- epilogue: O / l, bf16
+            *xslot(2, half) = l;
+            named_bar_sync(bar_id, 32 * NSP);
+            l = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
             ok = mbar_wait(&ofinal[t], 0) && ok;
             tc_fence_after();
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
-                                 ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D;
+                                 ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D + half * OCOL;
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
+            for (int q = 0; q < OCOL / 32; ++q) {
                 float o[32];
-                tmem_ld32(lane_base + C::COL_O + t * D + 32 * q, o);
+                tmem_ld32(lane_base + ocol + 32 * q, o);
                 tmem_wait_ld();
                 if (row_valid) {
 #pragma unroll
