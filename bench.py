@@ -144,6 +144,18 @@ def kv_bytes(lens, Hkv, D, eb):
     return int(np.asarray(lens, np.int64).sum()) * Hkv * D * 2 * eb
 
 
+def decode_alg_flops(lens, Hq, D):
+    """CUDA-core FLOPs of one decode launch: for every cached token and q
+    head, q.k and p.v over D dims, 2 FLOP per multiply-add."""
+    return 4 * D * Hq * int(np.asarray(lens, np.int64).sum())
+
+
+def alu_peak(sm_mhz):
+    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per
+    clock, at the SM clock sampled during the timed region."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def decode_alg_bytes(lens, Hq, Hkv, D, eb):
     lens = np.asarray(lens, np.int64)
     B = len(lens)
@@ -319,6 +331,7 @@ def run_ours(args, rank, world, device):
     kvb = sum(kv_bytes(ds.plan.decode_lens, Hkv, D, eb) for ds in timed)
     seqsteps = sum(ds.B for ds in timed)
     algb = [decode_alg_bytes(ds.plan.decode_lens, Hq, Hkv, D, eb) for ds in timed if ds.B]
+    algf = [decode_alg_flops(ds.plan.decode_lens, Hq, D) for ds in timed if ds.B]
     flags = ops.get_last_device_error()
     if flags:
         raise RuntimeError(f"device status word {flags:#x} after the timed steps")
@@ -357,7 +370,7 @@ def run_ours(args, rank, world, device):
         e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
         e2e = {"ms": e2e_ms, "h2d": h2d / len(hsteps), "d2h": d2h / len(hsteps), "kvb": kvb}
 
-    return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb,
+    return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb, algf=algf,
                 launches=launches, clocks=clk.summary(), e2e=e2e, plan_ms=t_plan * 1e3, tr=tr, plans=plans,
                 k_cache=k_cache, v_cache=v_cache, Hq=Hq, Hkv=Hkv, D=D, eb=eb, fp8=fp8, scale=scale,
                 k_scale=k_scale, v_scale=v_scale, q=q, pool=pool)
@@ -462,6 +475,7 @@ def run_mixed(args, rank, world, device):
                      dc.num_blocks + pc.k_cache.shape[0])
     return dict(tot_ms=sum(step_ms), step_ms=step_ms, dec_ms=dec_ms, kvb=kvb_step * args.steps,
                 seqsteps=dc.B * args.steps, algb=[decode_alg_bytes(dc.seq_lens, dc.Hq, dc.Hkv, dc.D, 2)] * args.steps,
+                algf=[decode_alg_flops(dc.seq_lens, dc.Hq, dc.D)] * args.steps,
                 launches=launches, clocks=clk.summary(), e2e=None, plan_ms=0.0, tr=tr, plans=None, fp8=False,
                 prefill={"ms": sum(pre_ms) / len(pre_ms), "flops": prefill_flops(pc.cu_q, pc.prefix_lens, pc.Hq, pc.D),
                          "tokens": int(pc.cu_q[-1])})
@@ -621,7 +635,24 @@ def main():
         peak, peak_kind = peaks()
         dec_ms = sum(r["dec_ms"]) / len(r["dec_ms"])
         alg = sum(r["algb"]) / len(r["algb"])
+        flops = sum(r["algf"]) / len(r["algf"])
         achieved = alg / (dec_ms / 1e3) / 1e9
+        # the binding roof: HBM bytes or CUDA-core FLOPs (GQA 8 with an fp8
+        # cache does 16 FLOP per cached byte and is arithmetic-bound)
+        sm_mhz = (r["clocks"] or {}).get("sm_mhz") or 1965.0
+        apeak = alu_peak(sm_mhz)
+        alu_bound = flops / (apeak * 1e12) > alg / (peak * 1e9)
+        if alu_bound:
+            tfl = flops / (dec_ms / 1e3) / 1e12
+            roof = {"bound": "alu", "achieved": tfl, "peak": apeak, "unit": "TFLOP/s", "frac": tfl / apeak,
+                    "peak_kind": f"derived: 148 SMs x 128 fp32 lanes x 2 FLOP x {sm_mhz:.0f} MHz",
+                    "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak}
+        else:
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "peak_kind": f"{peak_kind} (copy bandwidth)"}
+        roof.update({"kernel": "pa_decode (decode + merge)",
+                     "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", args.workload),
+                     "alg_bytes_per_launch": alg, "alg_flops_per_launch": flops, "ms_per_launch": dec_ms})
         tr = r["tr"]
         line = {
             "metric": METRIC, "value": kvb / tot_s / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -630,10 +661,7 @@ def main():
             "data": "synthetic", "config": workload_config(args, tr),
             "seq_steps_per_s": seqsteps / tot_s,
             "pct_of_hbm_peak": 100.0 * (kvb / tot_s / 1e9) / peak,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "peak_kind": f"{peak_kind} (copy bandwidth)", "kernel": "pa_decode (decode + merge)",
-                         "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", args.workload),
-                         "alg_bytes_per_launch": alg, "ms_per_launch": dec_ms},
+            "roofline": roof,
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
             "host_plan_ms_per_step": r["plan_ms"],
