@@ -31,7 +31,9 @@
 //    the other tile's softmax runs.
 //  * S_t(j+1) is issued only after O_t += P_t(j) V_j has completed (it
 //    overwrites P_t), so when softmax t sees S_t(j+1) the previous P.V is
-//    done and a rescale of its O row in TMEM is safe.
+//    done and a rescale of its O row in TMEM is safe.  The MMA warp issues,
+//    per tile in turn, P.V as soon as P arrives and then the tile's next S,
+//    so a tile never waits for the other tile's softmax.
 //  * Softmax applies the causal mask only on tiles that reach past the
 //    row's position, moves the running max only when it grows by more than
 //    8 (log2 units), and computes P with one packed FMA and one MUFU.EX2
@@ -205,33 +207,35 @@ __global__ void __launch_bounds__(C::NT, 1)
             }
         }
     } else if (w == C::W_MMA) {
-        // ---- MMA issue, per K/V tile j: S_t(j) for both query tiles, then
-        // O_t += P_t(j) V_j as each softmax warpgroup hands over P_t(j)
+        // ---- MMA issue, software-pipelined per query tile: O_t += P_t(j) V_j
+        // as soon as softmax t hands over P_t(j), then S_t(j+1) = Q_t K_{j+1}^T
+        // as soon as that P.V has completed (S_t(j+1) overwrites P_t).  Tile
+        // 0's next scores never wait for tile 1's softmax, and tile 1 stays
+        // half a step behind tile 0, so the two softmaxes use MUFU in turns.
         constexpr uint32_t idS = idesc_bf16_f32(128, KT, false);
         constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
-        for (int j = 0; j < ntiles; ++j) {
-            const int s = j % NS;
-            ok = mbar_wait(&kfull[s], (j / NS) & 1) && ok;
+        auto issue_s = [&](int t, int jj) {
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t q0 = smem_addr(sQ + t * C::QTILE), k0 = smem_addr(sK + (jj % NS) * C::KTILE);
 #pragma unroll
-            for (int t = 0; t < NQ; ++t) {
-                if (j < ntl[t]) {
-                    // P_t(j-1), in S_t's columns, has been consumed
-                    if (j > 0) ok = mbar_wait(&odone[t], (j - 1) & 1) && ok;
-                    if (lane == 0) {
-                        tc_fence_after();
-                        const uint32_t q0 = smem_addr(sQ + t * C::QTILE), k0 = smem_addr(sK + s * C::KTILE);
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            tc_mma_bf16(tmem + t * KT, smem_desc_sw128(q0 + (kk / 4) * C::QATOM + (kk % 4) * 32, 16, 1024),
-                                        smem_desc_sw128(k0 + (kk / 4) * C::KATOM + (kk % 4) * 32, 16, 1024), idS,
-                                        kk > 0);
-                        tc_commit(&sfull[t]);
-                    }
-                    __syncwarp();
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc_mma_bf16(tmem + t * KT, smem_desc_sw128(q0 + (kk / 4) * C::QATOM + (kk % 4) * 32, 16, 1024),
+                                smem_desc_sw128(k0 + (kk / 4) * C::KATOM + (kk % 4) * 32, 16, 1024), idS, kk > 0);
+                tc_commit(&sfull[t]);
             }
-            if (lane == 0) tc_commit(&kempty[s]);
             __syncwarp();
+        };
+        if (ntiles > 0) {
+            ok = mbar_wait(&kfull[0], 0) && ok;
+#pragma unroll
+            for (int t = 0; t < NQ; ++t)
+                if (ntl[t] > 0) issue_s(t, 0);
+            if (lane == 0) tc_commit(&kempty[0]);
+            __syncwarp();
+        }
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % NS, jn = j + 1, sn = jn % NS;
             ok = mbar_wait(&vfull[s], (j / NS) & 1) && ok;
             const int kv0 = j * KT;
             if (kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
@@ -245,6 +249,7 @@ __global__ void __launch_bounds__(C::NT, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
             }
+            bool kready = false;  // K tile j+1 has landed
 #pragma unroll
             for (int t = 0; t < NQ; ++t) {
                 if (j < ntl[t]) {
@@ -262,9 +267,22 @@ __global__ void __launch_bounds__(C::NT, 1)
                     }
                     __syncwarp();
                 }
+                if (jn < ntl[t]) {
+                    if (!kready) {
+                        ok = mbar_wait(&kfull[sn], (jn / NS) & 1) && ok;
+                        kready = true;
+                    }
+                    ok = mbar_wait(&odone[t], j & 1) && ok;  // P_t(j) consumed
+                    issue_s(t, jn);
+                }
             }
             if (lane == 0) tc_commit(&vempty[s]);
             __syncwarp();
+            if (jn < ntiles) {
+                if (!kready) ok = mbar_wait(&kfull[sn], (jn / NS) & 1) && ok;
+                if (lane == 0) tc_commit(&kempty[sn]);  // after every S(j+1) above
+                __syncwarp();
+            }
         }
         // every MMA of this CTA has completed before TMEM is released
         if (lane == 0) tc_commit(mma_done);
