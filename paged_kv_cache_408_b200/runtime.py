@@ -19,6 +19,10 @@ Sources (by page and section):
   conversation whose cache is later recomputed.
 * same page, What it means in production -- max_num_seqs and
   max_num_batched_tokens bound the batch.
+* "Production Serving: Continuous Batching and PagedAttention", The Build,
+  Step 8 "Prefix caching" -- a cache from full-page token prefixes to the
+  pages that hold them; a new prompt looks up its longest cached full-page
+  prefix, shares those pages (refcount + 1) and only computes the rest.
 
 Readings where the pages are silent: the preempted sequence is the most
 recently admitted running one; admission needs the blocks of the request's
@@ -34,7 +38,7 @@ kernels.
 from __future__ import annotations
 
 import math
-from collections import deque
+from collections import OrderedDict, deque
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -59,15 +63,21 @@ class BlockAllocator:
             raise ValueError("order must be a permutation of the pool")
         self.ref = np.zeros(self.num_blocks, np.int32)
         self.copies_emitted = 0
+        self.cache: PrefixCache | None = None  # attached by PrefixCache
 
     @property
     def num_free(self) -> int:
-        return len(self.free_list)
+        """Blocks an allocation can take: the free list plus cached blocks
+        that no sequence holds (evicted on demand)."""
+        return len(self.free_list) + (self.cache.num_evictable if self.cache else 0)
 
     def alloc(self) -> int:
-        if not self.free_list:
+        if self.free_list:
+            b = self.free_list.pop()
+        elif self.cache is not None and self.cache.num_evictable:
+            b = self.cache.evict()
+        else:
             raise OutOfBlocksError()
-        b = self.free_list.pop()
         self.ref[b] = 1
         return b
 
@@ -81,7 +91,123 @@ class BlockAllocator:
             raise RuntimeError(f"decref of free block {b}")
         self.ref[b] -= 1
         if self.ref[b] == 0:
-            self.free_list.append(b)
+            if self.cache is not None and self.cache.holds(b):
+                self.cache.park(b)  # stays cached until a lookup revives it or space is needed
+            else:
+                self.free_list.append(b)
+
+
+# ------------------------------------------------------------ prefix cache
+class PrefixCache:
+    """Full-block token prefixes -> physical blocks ("Production Serving:
+    Continuous Batching and PagedAttention", Step 8 "Prefix caching").
+
+    The pages key a dict by the token tuple of every full-page prefix.  Here
+    the key of block i of a prompt is (block holding tokens [0, 16 i) -- or
+    -1 for i = 0 --, the 16 token ids of block i): the same identity, since
+    the parent block stands for its whole prefix, without keys that grow with
+    the prefix.  A lookup walks the prompt block by block from the start and
+    returns the longest cached full-block prefix; its blocks are shared
+    (refcount + 1).
+
+    A cached block that no sequence holds any more is not freed: it waits in
+    LRU order (least recently released first) for a lookup to revive it, and
+    is evicted -- key removed, together with every cached block below it,
+    whose key names it -- only when an allocation finds the free list empty.
+    Sequences release their blocks last-to-first, so a prefix's deepest
+    blocks are evicted first.
+    """
+
+    def __init__(self, allocator: BlockAllocator):
+        self.alloc = allocator
+        allocator.cache = self
+        self.block_of: dict[tuple, int] = {}   # key -> block
+        self.key_of: dict[int, tuple] = {}     # block -> key
+        self.children: dict[int, set] = {}    # block -> cached blocks keyed under it
+        self.lru: OrderedDict[int, None] = OrderedDict()  # cached, refcount 0
+        self.hits = 0      # blocks shared by lookups
+        self.evictions = 0
+
+    @property
+    def num_evictable(self) -> int:
+        return len(self.lru)
+
+    def holds(self, b: int) -> bool:
+        return b in self.key_of
+
+    def park(self, b: int) -> None:
+        self.lru[b] = None
+
+    def _keys(self, tokens):
+        tokens = np.asarray(tokens)
+        for i in range(len(tokens) // BLOCK_SIZE):
+            yield tuple(int(t) for t in tokens[i * BLOCK_SIZE:(i + 1) * BLOCK_SIZE])
+
+    def peek(self, tokens) -> int:
+        """Blocks a lookup of ``tokens`` would share (no side effects)."""
+        parent, n = -1, 0
+        for blk in self._keys(tokens):
+            b = self.block_of.get((parent, blk))
+            if b is None:
+                break
+            parent, n = b, n + 1
+        return n
+
+    def match(self, tokens) -> tuple[int, list]:
+        """Longest cached full-block prefix of ``tokens``: (tokens covered,
+        blocks), each block's refcount incremented (revived if parked)."""
+        blocks, parent = [], -1
+        for blk in self._keys(tokens):
+            b = self.block_of.get((parent, blk))
+            if b is None:
+                break
+            blocks.append(b)
+            parent = b
+        for b in blocks:
+            if self.alloc.ref[b] == 0:
+                del self.lru[b]
+                self.alloc.ref[b] = 1
+            else:
+                self.alloc.incref(b)
+        self.hits += len(blocks)
+        return BLOCK_SIZE * len(blocks), blocks
+
+    def insert(self, tokens, block_table) -> None:
+        """Register the full blocks of a computed prompt: ``tokens`` are the
+        positions whose K/V are in ``block_table``'s blocks."""
+        parent = -1
+        for i, blk in enumerate(self._keys(tokens)):
+            key = (parent, blk)
+            b = self.block_of.get(key)
+            if b is None:
+                b = int(block_table[i])
+                if b in self.key_of:  # this block already caches another prefix
+                    return
+                self.block_of[key] = b
+                self.key_of[b] = key
+                if parent >= 0:
+                    self.children.setdefault(parent, set()).add(b)
+            parent = b
+
+    def _forget(self, b: int) -> None:
+        """Drop b's key and, recursively, the keys of the blocks under it;
+        those of them that no sequence holds go back to the free list."""
+        for c in self.children.pop(b, ()):
+            self._forget(c)
+            if c in self.lru:
+                del self.lru[c]
+                self.alloc.free_list.append(c)
+        key = self.key_of.pop(b)
+        del self.block_of[key]
+        if key[0] >= 0 and key[0] in self.children:
+            self.children[key[0]].discard(b)
+
+    def evict(self) -> int:
+        """Take the least recently released cached block for a new use."""
+        b, _ = self.lru.popitem(last=False)
+        self._forget(b)
+        self.evictions += 1
+        return b
 
 
 # ---------------------------------------------------------------- sequences
@@ -108,6 +234,7 @@ class Sequence:
     status: str = WAITING
     admitted_at: int = -1
     preemptions: int = 0
+    tokens: np.ndarray | None = None  # prompt token ids (needed only for prefix caching)
 
     @property
     def in_prefill(self) -> bool:
@@ -155,7 +282,10 @@ class KVManager:
         return child
 
     def release(self, seq: Sequence) -> None:
-        for b in seq.block_table:
+        # table order, as the pages return pages; with a prefix cache, deepest
+        # first, so that its LRU evicts a prefix's leaves before its root
+        order = seq.block_table if self.alloc.cache is None else reversed(seq.block_table)
+        for b in order:
             self.alloc.decref(b)
         seq.block_table = []
 
@@ -204,6 +334,7 @@ class SchedulerConfig:
     max_chunk: int = 8192          # longest prefill chunk
     max_blocks_per_seq: int = 512  # width of the uploaded block tables
     watermark: float = 0.01        # fraction of the pool kept free at admission
+    prefix_cache: bool = False     # share cached full-block prompt prefixes
 
 
 class Scheduler:
@@ -221,6 +352,7 @@ class Scheduler:
         self.admit_counter = 0
         self.num_preemptions = 0
         self.watermark_blocks = int(math.ceil(self.cfg.watermark * allocator.num_blocks))
+        self.cache = PrefixCache(allocator) if self.cfg.prefix_cache else None
 
     # -- requests
     def add_request(self, seq: Sequence) -> None:
@@ -281,8 +413,18 @@ class Scheduler:
         plan.preempted.append(victim.seq_id)
         return victim
 
+    def _lookup_tokens(self, seq: Sequence):
+        """Prompt positions a prefix-cache lookup may cover: all but the last
+        one, which must be computed to continue the sequence."""
+        if self.cache is None or seq.tokens is None or seq.num_cached or seq.block_table:
+            return None
+        return np.asarray(seq.tokens)[:max(0, seq.prefill_end - 1)]
+
     def _can_admit(self, seq: Sequence) -> bool:
         need = blocks_for(seq.prefill_end)
+        toks = self._lookup_tokens(seq)
+        if toks is not None:
+            need -= self.cache.peek(toks)  # shared blocks are not allocated
         return self.alloc.num_free >= need + self.watermark_blocks
 
     def _table(self, seqs) -> np.ndarray:
@@ -336,6 +478,9 @@ class Scheduler:
             if s.seq_id in plan.preempted or not self._can_admit(s):
                 break  # a sequence evicted in this step waits at least one step
             self.waiting.popleft()
+            toks = self._lookup_tokens(s)
+            if toks is not None:
+                s.num_cached, s.block_table = self.cache.match(toks)
             self.add_running(s)
             plan.admitted.append(s.seq_id)
             n = min(budget, s.prefill_end - s.num_cached, self.cfg.max_chunk)
@@ -391,6 +536,8 @@ class Scheduler:
             if s.num_cached >= s.prefill_end and s.fresh:
                 s.fresh = False
                 s.num_tokens = s.num_cached + 1  # the prompt's last position samples a token
+                if self.cache is not None and s.tokens is not None:
+                    self.cache.insert(np.asarray(s.tokens)[:s.num_cached], s.block_table)
         self.step_no += 1
 
     # -- accounting
@@ -407,8 +554,10 @@ class Scheduler:
 
 # ------------------------------------------------------------ invariants
 def check_invariants(sched: Scheduler) -> None:
-    """refcount[p] == number of block tables referencing p; free list and
-    referenced blocks partition the pool; no block is free and referenced."""
+    """refcount[p] == number of block tables referencing p; the free list,
+    the parked cached blocks and the referenced blocks partition the pool;
+    every cached key names a block that is referenced or parked, and its
+    parent is cached too."""
     a = sched.alloc
     count = np.zeros(a.num_blocks, np.int64)
     for s in sched.running:
@@ -424,5 +573,15 @@ def check_invariants(sched: Scheduler) -> None:
     free[a.free_list] = True
     if len(a.free_list) != int(free.sum()):
         raise AssertionError("duplicate entries in the free list")
-    if np.any(free & (a.ref > 0)) or np.any(~free & (a.ref == 0)):
-        raise AssertionError("free list and referenced blocks do not partition the pool")
+    parked = np.zeros(a.num_blocks, bool)
+    if a.cache is not None:
+        parked[list(a.cache.lru)] = True
+        for b, key in a.cache.key_of.items():
+            if free[b] or (a.ref[b] == 0 and not parked[b]):
+                raise AssertionError(f"cached block {b} is free")
+            if a.cache.block_of.get(key) != b or (key[0] >= 0 and key[0] not in a.cache.key_of):
+                raise AssertionError(f"cache maps of block {b} disagree")
+        if any(b not in a.cache.key_of for b in a.cache.lru):
+            raise AssertionError("a parked block has no key")
+    if np.any(free & parked) or np.any((free | parked) & (a.ref > 0)) or np.any(~(free | parked) & (a.ref == 0)):
+        raise AssertionError("free list, parked cached blocks and referenced blocks do not partition the pool")
