@@ -189,6 +189,44 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               void *workspace, size_t workspace_bytes, const pa_cache_desc *desc, pa_stream_t stream);
 
 /*
+ * pa_decode_cascade -- pa_decode for a batch whose sequences all begin with
+ * the same prefix_blocks physical blocks (a shared prompt; sequences forked
+ * from one parent).  [PS] Step 6 defines the result (per query head, over
+ * every cached token of the sequence), which equals pa_decode's; the pages
+ * state that such blocks are shared ("Production Serving: Continuous
+ * Batching and PagedAttention", Step 4; "Continuous batching and
+ * PagedAttention", PagedAttention: KV cache memory) but give no kernel for
+ * reading them once, so the split below is this library's.
+ *
+ * The keys of each sequence split into the shared prefix [0, 16*prefix_blocks)
+ * and its own suffix.  The prefix is attended once per kv head for every
+ * sequence at the same time (its K/V read once, all sequences' queries as
+ * the rows of a tensor-core attention; an fp8 prefix is first widened to
+ * bf16 exactly, into the workspace), each suffix by the decode kernel, and
+ * the two are combined by the split-K log-sum-exp merge.
+ *
+ * Arguments as pa_decode (balanced split), plus:
+ *   prefix_blocks  number of leading block-table entries that every row
+ *                  shares: entries 0..prefix_blocks-1 of every row must equal
+ *                  those of row 0 (not checked; row 0's are used).  0 runs
+ *                  pa_decode.  Every seq_lens[b] must be >= 16*prefix_blocks
+ *                  (checked on the device: PA_DEVERR_BAD_LEN).
+ *   workspace      at least pa_decode_cascade_workspace_size() bytes,
+ *                  256-byte aligned, no initialisation needed (every call
+ *                  writes all it reads).  Calls sharing one workspace must
+ *                  not overlap on the GPU.
+ * head_dim 64 or 128; bf16 or fp8 E4M3 cache (with k_scale, v_scale).
+ */
+int pa_decode_cascade_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                                     int32_t prefix_blocks, const pa_cache_desc *desc, size_t *bytes);
+
+int pa_decode_cascade(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *seq_lens, int32_t num_seqs,
+                      int32_t max_blocks_per_seq, int32_t num_q_heads, float scale, const float *k_scale,
+                      const float *v_scale, int32_t prefix_blocks, void *workspace, size_t workspace_bytes,
+                      const pa_cache_desc *desc, pa_stream_t stream);
+
+/*
  * pa_prefill_chunk -- causal attention of prompt chunks over their paged
  * prefixes (chunked prefill).
  * [CB] "How the scheduler works": a long prompt is cut into chunks that fit

@@ -151,6 +151,49 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
     return from_cuda(pa::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 
+int pa_decode_cascade_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_blocks_per_seq,
+                                     int32_t prefix_blocks, const pa_cache_desc *desc, size_t *bytes) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || prefix_blocks < 0 ||
+        prefix_blocks > max_blocks_per_seq)
+        return PA_ERR_INVALID_ARG;
+    *bytes = pa::cascade_ws_bytes(num_seqs, num_q_heads, desc->num_kv_heads, desc->head_dim, max_blocks_per_seq,
+                                  prefix_blocks, desc->dtype == PA_DTYPE_FP8_E4M3);
+    return PA_OK;
+}
+
+int pa_decode_cascade(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *seq_lens, int32_t num_seqs,
+                      int32_t max_blocks_per_seq, int32_t num_q_heads, float scale, const float *k_scale,
+                      const float *v_scale, int32_t prefix_blocks, void *workspace, size_t workspace_bytes,
+                      const pa_cache_desc *desc, pa_stream_t stream) {
+    int rc = check_desc(desc);
+    if (rc != PA_OK) return rc;
+    if (num_seqs < 0 || num_seqs > kMaxSeqs || max_blocks_per_seq <= 0 || num_q_heads <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (prefix_blocks < 0 || prefix_blocks > max_blocks_per_seq) return PA_ERR_INVALID_ARG;
+    if (prefix_blocks == 0)  // nothing shared: plain decode
+        return pa_decode(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
+                         num_q_heads, scale, k_scale, v_scale, 0, workspace, workspace_bytes, desc, stream);
+    if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (desc->num_kv_heads > pa::kMaxDecodeKvHeads) return PA_ERR_UNSUPPORTED;
+    const int G = num_q_heads / desc->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
+    const bool fp8 = desc->dtype == PA_DTYPE_FP8_E4M3;
+    if (fp8 && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+    const size_t need = pa::cascade_ws_bytes(num_seqs, num_q_heads, desc->num_kv_heads, desc->head_dim,
+                                             max_blocks_per_seq, prefix_blocks, fp8);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return PA_ERR_WORKSPACE;
+    pa::DecodeArgs a{out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, max_blocks_per_seq,
+                     num_q_heads, desc->num_kv_heads, desc->head_dim, desc->num_blocks, scale, k_scale, v_scale,
+                     0, 0, nullptr, nullptr, nullptr, fp8, status_word_ptr(), prefix_blocks};
+    return from_cuda(pa::launch_decode_cascade(a, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const int32_t *prefix_lens,
                      const int32_t *block_tables, int32_t num_chunks, int32_t max_blocks_per_seq,
                      int32_t num_q_heads, int32_t max_q_len, int32_t total_q_tokens, const void *k_cache,

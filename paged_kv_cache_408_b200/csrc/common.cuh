@@ -150,6 +150,13 @@ PA_DEVICE float ex2(float x) {
     return y;
 }
 
+// log2(x) with the hardware approximation (MUFU.LG2).
+PA_DEVICE float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Two bf16 packed in one 32-bit word -> (low element, high element) as fp32.
 // bf16 is the upper half of a binary32, so widening is a shift / mask.
 PA_DEVICE float2 bf16x2_to_float2(uint32_t w) {

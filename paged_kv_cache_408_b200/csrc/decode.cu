@@ -71,12 +71,6 @@ constexpr int kSegmentCost = 2;            // balanced split: cost units charged
 constexpr size_t kRingBytes = 192 * 1024;  // K/V staging rings of all warps of an SM
 constexpr unsigned kFull = 0xffffffffu;
 
-PA_DEVICE float lg2(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 template <int D_, int G_, bool FP8_>
 struct Cfg {
     static constexpr int D = D_, G = G_;
@@ -323,7 +317,7 @@ struct Producer {
     uint32_t issued;
 
     PA_DEVICE int load32(const DecodeArgs &a, const Item &it, int lane, int off) {
-        const int32_t *row = a.block_tables + (size_t)it.b * a.max_blocks + it.blk0;
+        const int32_t *row = a.block_tables + (size_t)it.b * a.max_blocks + a.prefix_blocks + it.blk0;
         return (off + lane < it.nblk) ? row[off + lane] : -1;
     }
 
@@ -446,14 +440,14 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     // ---- lengths, then exclusive scans over sequences: the balanced split
     // needs each sequence's offset in the line (Hkv segments of cost units),
     // the fixed one the numbers of full partitions and of ragged tails.
-    const int cap = a.max_blocks * 16;
+    const int cap = a.max_blocks * 16, skip = a.prefix_blocks * 16;  // cascade: attend tokens [skip, len)
     for (int b = tid; b < B; b += C::NT) {
         int len = a.seq_lens[b];
-        if (len < 0 || len > cap) {
+        if (len < skip || len > cap) {
             flag_error(a.err, PA_DEVERR_BAD_LEN);
-            len = 0;
+            len = skip;
         }
-        s_len[b] = len;
+        s_len[b] = len - skip;
     }
     if (lane < C::NSTAGE) mbar_init(&bars[w * C::NSTAGE + lane], 1);
     fence_mbar_init();
@@ -518,11 +512,16 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
         sc.total = (sc.NF + s_pre1[B]) * Hkv;
         sc.S = 0;
     }
-    // empty sequences produce all-zero rows (no item covers them)
+    // empty sequences produce all-zero rows (no item covers them); in a
+    // cascade their output is the shared-prefix piece alone
     for (int b = blockIdx.x; b < B; b += gridDim.x)
-        if (s_len[b] == 0)
-            for (int i = tid; i < a.Hq * D; i += C::NT)
-                static_cast<__nv_bfloat16 *>(a.out)[(size_t)b * a.Hq * D + i] = __float2bfloat16_rn(0.f);
+        if (s_len[b] == 0) {
+            if (a.prefix_blocks)
+                for (int k = tid; k < Hkv; k += C::NT) a.ws_np[(size_t)b * Hkv + k] = 1;
+            else
+                for (int i = tid; i < a.Hq * D; i += C::NT)
+                    static_cast<__nv_bfloat16 *>(a.out)[(size_t)b * a.Hq * D + i] = __float2bfloat16_rn(0.f);
+        }
 
     const uint8_t *kc = static_cast<const uint8_t *>(a.k_cache);
     const uint8_t *vc = static_cast<const uint8_t *>(a.v_cache);
@@ -676,7 +675,7 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
         group_merge<LPT, LPT, G, P2, C::NCH == 2>(m, l, acc2);
 
         // every group now holds the warp's result; group 0 writes it
-        if (it.npieces == 1) {
+        if (it.npieces == 1 && !a.prefix_blocks) {
             if (g == 0) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
@@ -699,11 +698,13 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
         } else {
             // ---- split-K: this piece's normalised output and log2-sum-exp;
             // piece 0 also records how many pieces the merge kernel combines
+            // (in a cascade the pieces follow the shared-prefix piece 0)
+            const int piece = it.piece + (a.prefix_blocks ? 1 : 0);
             if (g == 0) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
-                    float *dst = a.ws_o + ((row0 + (h ^ sh)) * a.max_parts + it.piece) * D;
+                    float *dst = a.ws_o + ((row0 + (h ^ sh)) * a.max_parts + piece) * D;
 #pragma unroll
                     for (int c = 0; c < C::NCH; ++c) {
                         float4 *d4 = reinterpret_cast<float4 *>(dst + choff[c] * 8);
@@ -713,10 +714,11 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
                                             acc2[h][4 * c + 3].x * inv, acc2[h][4 * c + 3].y * inv);
                     }
                     if (sub == 0)  // sub 0 has sh == 0: slot h is head h
-                        a.ws_lse[(row0 + h) * a.max_parts + it.piece] = (l[h] > 0.f) ? m[h] + lg2(l[h]) : -INFINITY;
+                        a.ws_lse[(row0 + h) * a.max_parts + piece] = (l[h] > 0.f) ? m[h] + lg2(l[h]) : -INFINITY;
                 }
             }
-            if (lane == 0 && it.piece == 0) a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces;
+            if (lane == 0 && it.piece == 0)
+                a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces + (a.prefix_blocks ? 1 : 0);
         }
         it = nx;
         have = have_nx;
@@ -768,7 +770,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
             load_o(u, v[u]);
         }
     if (len <= 0 || len > a.max_blocks * 16) return;  // empty or rejected: the decode kernel wrote the row
-    if (np <= 1) return;                               // one piece: the decode kernel wrote the row
+    if (np <= (a.prefix_blocks ? 0 : 1)) return;       // one piece: the decode kernel wrote the row
     if (np > a.max_parts) {
         if (lane == 0) flag_error(a.err, PA_DEVERR_BAD_LEN);
         return;

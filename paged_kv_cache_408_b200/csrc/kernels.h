@@ -46,6 +46,8 @@ struct DecodeArgs {
     float *ws_lse;         // [B][Hq][max_parts]
     bool fp8;
     unsigned *err;
+    int prefix_blocks;     // cascade: the first prefix_blocks of every row are attended elsewhere (piece 0);
+                           // this launch attends the rest and writes it as pieces 1.. (0: off)
 };
 
 struct PrefillArgs {
@@ -57,6 +59,16 @@ struct PrefillArgs {
     const void *k_cache, *v_cache;
     float scale;
     unsigned *err;
+    // Shared-prefix mode (shared_len > 0): one "chunk" of total_q decode
+    // sequences (q is the decode q [total_q][Hq][D]) that all attend keys
+    // [0, shared_len) through block_tables row 0, without causal extension;
+    // instead of bf16 out, each row's normalised fp32 output and log2-sum-exp
+    // become split-K piece 0 of that row in ws_o / ws_lse.  Scores are scaled
+    // by k_scale[kv head] and outputs by v_scale[kv head] when given.
+    int shared_len;
+    const float *k_scale, *v_scale;
+    float *ws_o, *ws_lse;
+    int max_parts;
 };
 
 cudaError_t launch_write_kv(const WriteArgs &a, cudaStream_t st);
@@ -84,5 +96,13 @@ inline int decode_max_parts(int max_blocks, int partition_tokens) {
 size_t decode_ws_bytes(int B, int Hq, int D, int max_parts);
 // Points a.ws_np / a.ws_o / a.ws_lse into a workspace of decode_ws_bytes().
 void decode_ws_carve(void *base, int B, int Hq, int D, int max_parts, DecodeArgs &a);
+
+// Cascade decode (cascade.cu): rows share their first prefix_blocks blocks.
+// The workspace is the decode workspace for cascade_max_parts() pieces,
+// followed (fp8 caches) by an identity block table and bf16 copies of the
+// shared prefix of both caches.
+int cascade_max_parts(int max_blocks, int prefix_blocks);
+size_t cascade_ws_bytes(int B, int Hq, int Hkv, int D, int max_blocks, int prefix_blocks, bool fp8);
+cudaError_t launch_decode_cascade(const DecodeArgs &a, void *workspace, cudaStream_t st);
 
 }  // namespace pa

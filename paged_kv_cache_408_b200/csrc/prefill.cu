@@ -115,11 +115,14 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int i0 = blockIdx.x * (NQ * C::QPOS);
     pdl_trigger();
     pdl_wait();
-    const int q_start = a.cu_q[c];
-    const int clen = a.cu_q[c + 1] - q_start;
-    const int pfx = a.prefix_lens[c];
-    if (i0 >= clen) return;  // this CTA's positions lie past the chunk (uniform per CTA)
-    const int L = pfx + clen;
+    // causal chunk: rows are positions pfx + i, keys [0, pfx + i]; shared
+    // prefix: rows are sequences, keys [0, shared_len) for every row
+    const bool shared = a.shared_len > 0;
+    const int q_start = shared ? 0 : a.cu_q[c];
+    const int clen = shared ? a.total_q : a.cu_q[c + 1] - q_start;
+    const int pfx = shared ? a.shared_len : a.prefix_lens[c];
+    if (i0 >= clen) return;  // this CTA's rows lie past the chunk (uniform per CTA)
+    const int L = shared ? pfx : pfx + clen;  // keys of the sequence
     if (clen < 0 || pfx < 0 || L > a.max_blocks * 16 || q_start < 0 || q_start + clen > a.total_q) {
         if (tid == 0) flag_error(a.err, PA_DEVERR_BAD_LEN);
         return;
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     for (int t = 0; t < NQ; ++t) {
         const int first = i0 + t * C::QPOS;
         const int nv = max(0, min(C::QPOS, clen - first));
-        ntl[t] = nv > 0 ? (pfx + first + nv + KT - 1) / KT : 0;
+        ntl[t] = nv > 0 ? ((shared ? pfx : pfx + first + nv) + KT - 1) / KT : 0;
         ntiles = max(ntiles, ntl[t]);
     }
 
@@ -296,8 +299,8 @@ __global__ void __launch_bounds__(C::NT, 1)
         const int bar_id = 1 + t * 4 + (w % 4);  // named barrier of the NSP warps sharing these rows
         const int ip = i0 + t * C::QPOS + r / G;
         const bool row_valid = ip < clen;
-        const int pos = pfx + ip;
-        const float sl2 = a.scale * kLog2e;
+        const int pos = shared ? pfx - 1 : pfx + ip;  // last key the row attends
+        const float sl2 = a.scale * kLog2e * (a.k_scale ? a.k_scale[kvh] : 1.f);
         const uint32_t lane_base = tmem + ((uint32_t)((w & 3) * 32) << 16);
         const uint32_t scol = t * KT + half * SCOL;            // this thread's S columns
         const uint32_t pcol = t * KT + half * (SCOL / 2);      // its P words (two bf16 each)
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             mbar_arrive(&pfull[t]);
         }
         if (ntl[t] > 0) {
-            // ---- epilogue: O / l, bf16
+            // ---- epilogue: O / l, as bf16 output rows (or as split-K piece 0)
             *xslot(2, half) = l;
             named_bar_sync(bar_id, 32 * NSP);
             l = 0.f;
@@ -386,25 +389,46 @@ __global__ void __launch_bounds__(C::NT, 1)
             for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
             ok = mbar_wait(&ofinal[t], 0) && ok;
             tc_fence_after();
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
-                                 ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D + half * OCOL;
+            const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
+            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            if (shared) {
+                // split-K piece 0 of the row: normalised fp32 output and log2-sum-exp
+                const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;
+                float *wo = a.ws_o + grow * a.max_parts * D + half * OCOL;
 #pragma unroll
-            for (int q = 0; q < OCOL / 32; ++q) {
-                float o[32];
-                tmem_ld32(lane_base + ocol + 32 * q, o);
-                tmem_wait_ld();
-                if (row_valid) {
+                for (int q = 0; q < OCOL / 32; ++q) {
+                    float o[32];
+                    tmem_ld32(lane_base + ocol + 32 * q, o);
+                    tmem_wait_ld();
+                    if (row_valid) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint32_t wds[4];
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4 *>(wo + 32 * q + e) =
+                                make_float4(o[e] * inv * vs, o[e + 1] * inv * vs, o[e + 2] * inv * vs,
+                                            o[e + 3] * inv * vs);
+                    }
+                }
+                if (row_valid && half == 0) a.ws_lse[grow * a.max_parts] = (l > 0.f) ? m + lg2(l) : -INFINITY;
+            } else {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const __nv_bfloat162 bb =
-                                __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
-                            wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
+                for (int q = 0; q < OCOL / 32; ++q) {
+                    float o[32];
+                    tmem_ld32(lane_base + ocol + 32 * q, o);
+                    tmem_wait_ld();
+                    if (row_valid) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            uint32_t wds[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const __nv_bfloat162 bb =
+                                    __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
+                                wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + 32 * q + e) =
+                                make_uint4(wds[0], wds[1], wds[2], wds[3]);
                         }
-                        *reinterpret_cast<uint4 *>(dst + 32 * q + e) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
                     }
                 }
             }

@@ -286,10 +286,13 @@ def mixed_step(seed=0, n_decode=192, n_chunks=8, chunk=512):
     return dec, pre
 
 
-def prefix_share(seed=0, n_seqs=256, prefix=2048, suffix_lo=16, suffix_hi=512, Hq=64, Hkv=8, D=128):
+def prefix_share(seed=0, n_seqs=256, prefix=2048, suffix_lo=16, suffix_hi=512, Hq=64, Hkv=8, D=128, fp8=True):
     """256 sequences sharing one 2048-token prefix (the same physical blocks)
     plus per-sequence suffixes uniform in [16, 512]; 64/8 heads, head_dim
-    128; fp8 E4M3 cache with per-head fp32 scales."""
+    128; fp8 E4M3 cache with per-head fp32 scales (bf16 with ``fp8=False``).
+    A prefix that is not a whole number of blocks shares its partial last
+    block too (the block table entry), as a forked sequence does before its
+    first write."""
     rng = np.random.default_rng(30_000 + seed)
     suf = rng.integers(suffix_lo, suffix_hi + 1, n_seqs).astype(np.int32)
     pre_blocks = blocks_for(prefix)
@@ -307,10 +310,15 @@ def prefix_share(seed=0, n_seqs=256, prefix=2048, suffix_lo=16, suffix_hi=512, H
         pos += suf_blocks[i]
     lens = (prefix + suf).astype(np.int32)
     q = normal_bf16(rng, (n_seqs, Hq, D))
-    kc, ks = fp8_cache_from_normal(rng, (nb, Hkv, BLOCK_SIZE, D))
-    vc, vs = fp8_cache_from_normal(rng, (nb, Hkv, BLOCK_SIZE, D))
-    case = DecodeCase("256 seqs sharing a 2048-token prefix, 64/8 heads, d128, fp8", q, kc, vc, bt, lens,
-                      1.0 / math.sqrt(D), ks, vs)
+    if fp8:
+        kc, ks = fp8_cache_from_normal(rng, (nb, Hkv, BLOCK_SIZE, D))
+        vc, vs = fp8_cache_from_normal(rng, (nb, Hkv, BLOCK_SIZE, D))
+    else:
+        kc = normal_bf16(rng, (nb, Hkv, BLOCK_SIZE, D))
+        vc = normal_bf16(rng, (nb, Hkv, BLOCK_SIZE, D))
+        ks = vs = None
+    case = DecodeCase(f"{n_seqs} seqs sharing a {prefix}-token prefix, {Hq}/{Hkv} heads, d{D}, "
+                      f"{'fp8' if fp8 else 'bf16'}", q, kc, vc, bt, lens, 1.0 / math.sqrt(D), ks, vs)
     case.extra["free_blocks"] = perm[pos:].copy()
     case.extra["shared_blocks"] = shared.copy()
     return case

@@ -25,6 +25,7 @@ DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_LEN, DEVERR_BAD_PAIR, DEVERR_TIMEO
 EXPORTED = (
     "pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_size", "pa_decode", "pa_prefill_chunk",
     "pa_get_last_device_error", "pa_status_string", "pa_version", "pa_decode_noalloc",
+    "pa_decode_cascade_workspace_size", "pa_decode_cascade",
 )
 
 
@@ -59,6 +60,9 @@ def lib():
                                        C.POINTER(CacheDesc), p]
         L.pa_get_last_device_error.argtypes = [C.POINTER(C.c_uint32), p]
         L.pa_decode_noalloc.argtypes = [p, p, p, p, p, p, i32, i32, i32, f32, p, p, i32, C.POINTER(CacheDesc), p]
+        L.pa_decode_cascade_workspace_size.argtypes = [i32, i32, i32, i32, C.POINTER(CacheDesc), C.POINTER(sz)]
+        L.pa_decode_cascade.argtypes = [p, p, p, p, p, p, i32, i32, i32, f32, p, p, i32, p, sz,
+                                        C.POINTER(CacheDesc), p]
         L.pa_status_string.argtypes = [C.c_int]
         L.pa_status_string.restype = C.c_char_p
         for f in EXPORTED:
@@ -226,6 +230,45 @@ def decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, scale, k_sc
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), B,
         block_tables.shape[1], Hq, float(scale), _ptr(ks), _ptr(vs), int(partition_tokens), C.byref(desc),
         _stream(stream)))
+
+
+def cascade_workspace_size(num_seqs, num_q_heads, max_blocks_per_seq, prefix_blocks, k_cache) -> int:
+    desc = cache_desc(k_cache)
+    out = C.c_size_t(0)
+    _check("pa_decode_cascade_workspace_size", lib().pa_decode_cascade_workspace_size(
+        int(num_seqs), int(num_q_heads), int(max_blocks_per_seq), int(prefix_blocks), C.byref(desc), C.byref(out)))
+    return int(out.value)
+
+
+def alloc_cascade_workspace(num_seqs, num_q_heads, max_blocks_per_seq, prefix_blocks, k_cache):
+    """Caller-side helper: a torch buffer large enough for pa_decode_cascade
+    (no particular contents needed)."""
+    n = cascade_workspace_size(num_seqs, num_q_heads, max_blocks_per_seq, prefix_blocks, k_cache)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=k_cache.device)
+
+
+def decode_cascade(out, q, k_cache, v_cache, block_tables, seq_lens, scale, prefix_blocks, workspace,
+                   k_scale=None, v_scale=None, stream=None):
+    """pa_decode_cascade: pa_decode for sequences whose first prefix_blocks
+    block-table entries are the same physical blocks in every row (the
+    shared prefix is attended once per kv head on the tensor cores)."""
+    desc = _caches(k_cache, v_cache)
+    dev = k_cache.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    _need(workspace, "workspace", None, dev)
+    B, Hq, D = q.shape
+    if out.shape != q.shape or D != desc.head_dim:
+        raise ValueError("out/q shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("block_tables must be [B, max_blocks] and seq_lens [B]")
+    ks, vs = _scales(desc, k_scale, v_scale, dev)
+    _check("pa_decode_cascade", lib().pa_decode_cascade(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), B,
+        block_tables.shape[1], Hq, float(scale), _ptr(ks), _ptr(vs), int(prefix_blocks), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), C.byref(desc), _stream(stream)))
 
 
 def prefill_chunk(out, q, cu_q_lens, prefix_lens, block_tables, k_cache, v_cache, scale, max_q_len,

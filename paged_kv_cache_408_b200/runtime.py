@@ -326,6 +326,18 @@ class StepPlan:
     def max_chunk(self) -> int:
         return int(np.diff(self.prefill_cu).max(initial=0))
 
+    @property
+    def shared_decode_blocks(self) -> int:
+        """Leading block-table entries that every decode sequence shares (the
+        same physical blocks, e.g. a forked prompt) and fills completely:
+        the prefix a cascade decode attends once for the whole batch."""
+        t = self.decode_tables
+        if len(t) == 0:
+            return 0
+        same = (t == t[0]).all(axis=0)
+        n = int(np.argmin(same)) if not same.all() else t.shape[1]
+        return min(n, int(self.decode_lens.min()) // BLOCK_SIZE)
+
 
 @dataclass
 class SchedulerConfig:
