@@ -200,6 +200,7 @@ class DeviceStep:
         self.T = len(plan.slots)
         self.B = plan.num_decode
         self.nchunks = len(plan.prefill_ids)
+        self.pb = 0  # shared prefix blocks attended by cascade decode (0: plain decode)
 
     def to(self, device, non_blocking=True):
         d = object.__new__(DeviceStep)
@@ -248,7 +249,10 @@ def run_ours(args, rank, world, device):
     pq = torch.randn((max(Pmax_tok, 1), Hq, D), generator=g, device=device).to(torch.bfloat16)
     pout = torch.empty_like(pq)
     maxb = plans[0].decode_tables.shape[1]
-    ws = ops.alloc_workspace(max(Bmax, 1), Hq, D, maxb, args.partition, device=device)
+    pbs = [cascade_blocks(p, args) for p in plans]
+    ws_bytes = max([ops.decode_workspace_size(max(Bmax, 1), Hq, D, maxb, args.partition)] +
+                   [ops.cascade_workspace_size(p.num_decode, Hq, maxb, pb, k_cache) for p, pb in zip(plans, pbs) if pb])
+    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     flush = L2Flush(torch, device)
     scale = 1.0 / math.sqrt(D)
     run_prefill = args.workload == "mixed"
@@ -264,11 +268,21 @@ def run_ours(args, rank, world, device):
         return n
 
     def decode(ds, qq, oo):
+        if ds.B and ds.pb:
+            ops.decode_cascade(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.tables, ds.lens, scale, ds.pb, ws,
+                               k_scale, v_scale)
+            return 4 if fp8 else 3  # (fp8 widening) + prefix attention + suffix decode + merge
         if ds.B:
             ops.decode(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.tables, ds.lens, scale, k_scale, v_scale, ws,
                        args.partition)
             return 2  # decode kernel + merge kernel
         return 0
+
+    def suffix_decode(ds, qq, oo):
+        # the suffix stage of a cascade step on its own: the same keys through
+        # the decode kernel (suffix tables and lengths), for its roofline
+        ops.decode(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.sfx_tables, ds.sfx_lens, scale, k_scale, v_scale, ws,
+                   0)
 
     def prefill(ds, pqq, poo):
         if run_prefill and ds.nchunks:
@@ -279,6 +293,13 @@ def run_ours(args, rank, world, device):
         return 0
 
     dsteps = [DeviceStep(p, torch, device) for p in plans]
+    for ds, pb in zip(dsteps, pbs):
+        ds.pb = pb
+        if pb:
+            st_ = np.full_like(ds.plan.decode_tables, -1)
+            st_[:, :st_.shape[1] - pb] = ds.plan.decode_tables[:, pb:]
+            ds.sfx_tables = torch.from_numpy(st_).to(device)
+            ds.sfx_lens = torch.from_numpy(ds.plan.decode_lens - 16 * pb).to(device)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
 
@@ -323,10 +344,36 @@ def run_ours(args, rank, world, device):
             decode(ds, q, out)
             e1.record(st)
         torch.cuda.synchronize()
+        sfx_ev = []
+        if any(ds.pb for ds in timed):
+            torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
+            for ds in timed:
+                if ds.B and ds.pb:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    flush()
+                    e0.record(st)
+                    suffix_decode(ds, q, out)
+                    e1.record(st)
+                    sfx_ev.append((e0, e1, ds))
+            torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
     dec_ms = [e0.elapsed_time(e1) for e0, e1 in dev_ev]
+    cascade = None
+    if sfx_ev:
+        n = len(sfx_ev)
+        lens_sfx = [ds.plan.decode_lens - 16 * ds.pb for _, _, ds in sfx_ev]
+        cascade = {
+            "steps": n, "prefix_blocks": sorted({int(ds.pb) for _, _, ds in sfx_ev}),
+            "call_ms": sum(e0.elapsed_time(e1) for (e0, e1), ds in zip(dev_ev, timed) if ds.B and ds.pb) / n,
+            "suffix_ms": sum(e0.elapsed_time(e1) for e0, e1, _ in sfx_ev) / n,
+            "prefix_flops": sum(4 * D * Hq * ds.B * 16 * ds.pb for _, _, ds in sfx_ev) / n,
+            "suffix_flops": sum(decode_alg_flops(x, Hq, D) for x in lens_sfx) / n,
+            "suffix_bytes": sum(decode_alg_bytes(x, Hq, Hkv, D, eb) for x in lens_sfx) / n,
+            "unique_bytes": sum(decode_alg_bytes(x, Hq, Hkv, D, eb) + 16 * ds.pb * Hkv * D * 2 * eb
+                                for x, (_, _, ds) in zip(lens_sfx, sfx_ev)) / n,
+        }
     tot_ms = sum(step_ms)
     kvb = sum(kv_bytes(ds.plan.decode_lens, Hkv, D, eb) for ds in timed)
     seqsteps = sum(ds.B for ds in timed)
@@ -340,6 +387,8 @@ def run_ours(args, rank, world, device):
     e2e = None
     if not args.no_e2e:
         hsteps = [DeviceStep(p, torch, device, pin=True) for p in plans[args.warmup:]]
+        for hs, pb in zip(hsteps, pbs[args.warmup:]):
+            hs.pb = pb
         hq = q.cpu().pin_memory()
         hk = new_k.cpu().pin_memory()
         hv = new_v.cpu().pin_memory()
@@ -372,6 +421,7 @@ def run_ours(args, rank, world, device):
 
     return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb, algf=algf,
                 launches=launches, clocks=clk.summary(), e2e=e2e, plan_ms=t_plan * 1e3, tr=tr, plans=plans,
+                cascade=cascade,
                 k_cache=k_cache, v_cache=v_cache, Hq=Hq, Hkv=Hkv, D=D, eb=eb, fp8=fp8, scale=scale,
                 k_scale=k_scale, v_scale=v_scale, q=q, pool=pool)
 
@@ -574,6 +624,7 @@ def workload_config(args, tr):
     return {"workload": tr.name, "trace": args.workload, "seqs": tr.sched.cfg.max_num_seqs, "q_heads": tr.Hq,
             "kv_heads": tr.Hkv, "head_dim": tr.D, "block_size": 16, "cache_dtype": "fp8_e4m3" if tr.fp8 else "bf16",
             "pool_blocks": tr.sched.alloc.num_blocks, "partition_tokens": args.partition or "balanced",
+            "kv_bytes": "logical: every decoded sequence's cached K/V (a shared prefix counts once per sequence)",
             "l2": "flushed between steps outside the timed events (256 MiB written, then 256 MiB read)", "parallelism": "replicas"}
 
 
@@ -594,6 +645,52 @@ def aggregate(tot_s, kv_bytes_done, seq_steps, world, device):
 
 
 
+def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload):
+    """Roofline of a cascade decode call (fp8 widening, prefix attention on
+    the tensor cores, suffix decode, merge).  The suffix stage is timed on
+    its own (the decode kernel over the suffix tables); the prefix stage is
+    the call minus that.  The line's roofline is the stage that takes
+    longer; both stages and the call's combined roof are listed."""
+    t_call, t_sfx = c["call_ms"] / 1e3, c["suffix_ms"] / 1e3
+    t_pre = max(t_call - t_sfx, 1e-9)
+    tpeak, tkind = tensor_peak()
+    pre_tfl = c["prefix_flops"] / t_pre / 1e12
+    prefix = {"bound": "tensor", "achieved": pre_tfl, "peak": tpeak, "unit": "TFLOP/s", "frac": pre_tfl / tpeak,
+              "peak_kind": tkind, "kernel": "prefill_kernel (shared-prefix mode) + fp8 widening",
+              "ms_per_launch": t_pre * 1e3, "alg_flops_per_launch": c["prefix_flops"],
+              "timing": "cascade call minus the suffix stage timed alone", "traffic": None}
+    if c["suffix_flops"] / (apeak * 1e12) > c["suffix_bytes"] / (hbm_peak * 1e9):
+        tfl = c["suffix_flops"] / t_sfx / 1e12
+        suffix = {"bound": "alu", "achieved": tfl, "peak": apeak, "unit": "TFLOP/s", "frac": tfl / apeak,
+                  "peak_kind": f"derived: 148 SMs x 128 fp32 lanes x 2 FLOP x {sm_mhz:.0f} MHz"}
+    else:
+        gbs = c["suffix_bytes"] / t_sfx / 1e9
+        suffix = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                  "peak_kind": f"{hbm_kind} (copy bandwidth)"}
+    suffix.update({"kernel": "decode_kernel + merge_kernel (suffix)", "ms_per_launch": t_sfx * 1e3,
+                   "alg_flops_per_launch": c["suffix_flops"], "alg_bytes_per_launch": c["suffix_bytes"],
+                   "timing": "decode call over the suffix tables, CUDA events",
+                   "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", workload + ":suffix")})
+    roof_s = (c["prefix_flops"] / (tpeak * 1e12) +
+              max(c["suffix_flops"] / (apeak * 1e12), c["suffix_bytes"] / (hbm_peak * 1e9)))
+    out = dict(suffix if t_sfx >= t_pre else prefix)
+    out["stages"] = {"prefix": prefix, "suffix": suffix,
+                     "call": {"ms_per_launch": t_call * 1e3, "roof_ms": roof_s * 1e3, "frac": roof_s / t_call,
+                              "unique_kv_bytes": c["unique_bytes"], "prefix_blocks": c["prefix_blocks"]}}
+    return out
+
+
+def cascade_blocks(plan, args):
+    """Shared prefix blocks a step's decode attends through cascade decode:
+    every row's leading table entries are the same physical blocks (forked
+    sequences), for a batch and prefix large enough to pay for the extra
+    launches; else 0 (plain decode)."""
+    if args.no_cascade:
+        return 0
+    pb = plan.shared_decode_blocks
+    return pb if plan.num_decode >= 8 and pb * 16 >= 256 else 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -606,6 +703,7 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cascade", action="store_true", help="plain decode even where rows share prefix blocks")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -653,6 +751,8 @@ def main():
         roof.update({"kernel": "pa_decode (decode + merge)",
                      "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", args.workload),
                      "alg_bytes_per_launch": alg, "alg_flops_per_launch": flops, "ms_per_launch": dec_ms})
+        if r.get("cascade"):
+            roof = cascade_roofline(r["cascade"], peak, peak_kind, apeak, sm_mhz, args.workload)
         tr = r["tr"]
         line = {
             "metric": METRIC, "value": kvb / tot_s / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -660,6 +760,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if not r["fp8"] else "fp8_e4m3",
             "data": "synthetic", "config": workload_config(args, tr),
             "seq_steps_per_s": seqsteps / tot_s,
+            "decode_path": "cascade" if r.get("cascade") else "decode",
             "pct_of_hbm_peak": 100.0 * (kvb / tot_s / 1e9) / peak,
             "roofline": roof,
             "gpu_launches": r["launches"],

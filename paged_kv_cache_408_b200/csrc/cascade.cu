@@ -8,9 +8,9 @@
 //   * the shared prefix is attended ONCE per kv head for all sequences: its
 //     K/V are read once and the queries of every sequence and head of the
 //     kv head form the rows of a dense attention on the tensor cores (the
-//     prefill kernel in its shared-prefix mode), giving split-K piece 0 of
-//     every row;
-//   * the decode kernel attends each suffix (pieces 1..);
+//     prefill kernel in its shared-prefix mode), split over key ranges so
+//     that it fills the SMs, giving split-K pieces 0..S-1 of every row;
+//   * the decode kernel attends each suffix (pieces S..);
 //   * the log-sum-exp merge combines the pieces (the same merge as split-K).
 // An fp8 prefix is first widened to bf16 (exactly: every E4M3 value is a
 // bf16 value) into workspace scratch with an identity block table; the
@@ -25,6 +25,7 @@ namespace pa {
 namespace {
 
 size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+constexpr int kNumSMs = 148;
 
 // Widen the prefix blocks of both caches (block_tables row 0) to bf16 into
 // [prefix_blocks][Hkv][16][D] scratch and write the identity table.  One
@@ -66,7 +67,9 @@ __global__ void __launch_bounds__(256) widen_prefix_kernel(const uint8_t *__rest
 
 }  // namespace
 
-int cascade_max_parts(int max_blocks, int prefix_blocks) { return decode_max_parts(max_blocks - prefix_blocks, 0) + 1; }
+int cascade_max_parts(int max_blocks, int prefix_blocks) {
+    return decode_max_parts(max_blocks - prefix_blocks, 0) + kMaxPrefixSplits;
+}
 
 size_t cascade_ws_bytes(int B, int Hq, int Hkv, int D, int max_blocks, int prefix_blocks, bool fp8) {
     size_t n = decode_ws_bytes(B, Hq, D, cascade_max_parts(max_blocks, prefix_blocks));
@@ -93,6 +96,15 @@ cudaError_t launch_decode_cascade(const DecodeArgs &d, void *workspace, cudaStre
     p.ws_o = a.ws_o;
     p.ws_lse = a.ws_lse;
     p.max_parts = a.max_parts;
+    // split the prefix's keys so that the prefix attention fills the SMs:
+    // CTAs per split = kv heads x query tiles of 256 rows (rows = sequences x
+    // group), at most one split per 128-key tile
+    {
+        const int ctas = a.Hkv * ((a.B * (a.Hq / a.Hkv) + 255) / 256);
+        const int tiles = (p.shared_len + 127) / 128;
+        p.key_splits = std::max(1, std::min({kNumSMs / std::max(ctas, 1), kMaxPrefixSplits, tiles}));
+    }
+    a.prefix_pieces = p.key_splits;
     cudaError_t e = cudaSuccess;
     if (a.fp8) {
         char *sc = static_cast<char *>(workspace) + decode_ws_bytes(a.B, a.Hq, a.D, a.max_parts);

@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     for (int b = blockIdx.x; b < B; b += gridDim.x)
         if (s_len[b] == 0) {
             if (a.prefix_blocks)
-                for (int k = tid; k < Hkv; k += C::NT) a.ws_np[(size_t)b * Hkv + k] = 1;
+                for (int k = tid; k < Hkv; k += C::NT) a.ws_np[(size_t)b * Hkv + k] = a.prefix_pieces;
             else
                 for (int i = tid; i < a.Hq * D; i += C::NT)
                     static_cast<__nv_bfloat16 *>(a.out)[(size_t)b * a.Hq * D + i] = __float2bfloat16_rn(0.f);
@@ -698,8 +698,8 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
         } else {
             // ---- split-K: this piece's normalised output and log2-sum-exp;
             // piece 0 also records how many pieces the merge kernel combines
-            // (in a cascade the pieces follow the shared-prefix piece 0)
-            const int piece = it.piece + (a.prefix_blocks ? 1 : 0);
+            // (in a cascade the pieces follow the shared prefix's pieces)
+            const int piece = it.piece + a.prefix_pieces;
             if (g == 0) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
@@ -718,7 +718,7 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
                 }
             }
             if (lane == 0 && it.piece == 0)
-                a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces + (a.prefix_blocks ? 1 : 0);
+                a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces + a.prefix_pieces;
         }
         it = nx;
         have = have_nx;

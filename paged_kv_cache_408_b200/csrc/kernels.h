@@ -46,8 +46,9 @@ struct DecodeArgs {
     float *ws_lse;         // [B][Hq][max_parts]
     bool fp8;
     unsigned *err;
-    int prefix_blocks;     // cascade: the first prefix_blocks of every row are attended elsewhere (piece 0);
-                           // this launch attends the rest and writes it as pieces 1.. (0: off)
+    int prefix_blocks;     // cascade: the first prefix_blocks of every row are attended elsewhere (pieces
+                           // 0..prefix_pieces-1); this launch attends the rest as the pieces after them (0: off)
+    int prefix_pieces;
 };
 
 struct PrefillArgs {
@@ -61,14 +62,17 @@ struct PrefillArgs {
     unsigned *err;
     // Shared-prefix mode (shared_len > 0): one "chunk" of total_q decode
     // sequences (q is the decode q [total_q][Hq][D]) that all attend keys
-    // [0, shared_len) through block_tables row 0, without causal extension;
-    // instead of bf16 out, each row's normalised fp32 output and log2-sum-exp
-    // become split-K piece 0 of that row in ws_o / ws_lse.  Scores are scaled
-    // by k_scale[kv head] and outputs by v_scale[kv head] when given.
+    // [0, shared_len) through block_tables row 0, without causal extension,
+    // split over key_splits ranges of whole key tiles (at most one range per
+    // tile); instead of bf16 out, each row's normalised fp32 output and
+    // log2-sum-exp over range z become split-K piece z of that row in ws_o /
+    // ws_lse.  Scores are scaled by k_scale[kv head] and outputs by
+    // v_scale[kv head] when given.
     int shared_len;
     const float *k_scale, *v_scale;
     float *ws_o, *ws_lse;
     int max_parts;
+    int key_splits;
 };
 
 cudaError_t launch_write_kv(const WriteArgs &a, cudaStream_t st);
@@ -101,6 +105,7 @@ void decode_ws_carve(void *base, int B, int Hq, int D, int max_parts, DecodeArgs
 // The workspace is the decode workspace for cascade_max_parts() pieces,
 // followed (fp8 caches) by an identity block table and bf16 copies of the
 // shared prefix of both caches.
+constexpr int kMaxPrefixSplits = 4;  // key ranges the shared prefix is split into
 int cascade_max_parts(int max_blocks, int prefix_blocks);
 size_t cascade_ws_bytes(int B, int Hq, int Hkv, int D, int max_blocks, int prefix_blocks, bool fp8);
 cudaError_t launch_decode_cascade(const DecodeArgs &a, void *workspace, cudaStream_t st);

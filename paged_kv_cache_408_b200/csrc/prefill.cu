@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     float *xch = reinterpret_cast<float *>(smem + C::OFF_X);  // [3][NQ][NSPLIT][128]: max (2 parities), sum
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.z, kvh = blockIdx.y;
+    const int c = a.shared_len > 0 ? 0 : blockIdx.z, kvh = blockIdx.y;
     const int i0 = blockIdx.x * (NQ * C::QPOS);
     pdl_trigger();
     pdl_wait();
@@ -128,6 +128,15 @@ __global__ void __launch_bounds__(C::NT, 1)
         return;
     }
     const int nalloc = (L + 15) >> 4;  // blocks of the sequence
+    // a shared prefix is split over its keys (grid z): this CTA attends key
+    // tiles [jt0, jt1) and writes split-K piece blockIdx.z of its rows
+    const int ks = shared ? (int)gridDim.z : 1, kz = shared ? (int)blockIdx.z : 0;
+    const int jt0 = shared ? kz * ((L + KT - 1) / KT) / ks : 0;
+    const int jt1 = shared ? (kz + 1) * ((L + KT - 1) / KT) / ks : 0;
+    if (shared && jt1 <= jt0) {  // more splits than key tiles
+        if (tid == 0) flag_error(a.err, PA_DEVERR_BAD_LEN);
+        return;
+    }
     const int32_t *bt = a.block_tables + (size_t)c * a.max_blocks;
     // K/V tiles each query tile needs (causal: up to its last valid row)
     int ntl[NQ], ntiles = 0;
@@ -135,7 +144,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     for (int t = 0; t < NQ; ++t) {
         const int first = i0 + t * C::QPOS;
         const int nv = max(0, min(C::QPOS, clen - first));
-        ntl[t] = nv > 0 ? ((shared ? pfx : pfx + first + nv) + KT - 1) / KT : 0;
+        ntl[t] = nv > 0 ? (shared ? jt1 - jt0 : (pfx + first + nv + KT - 1) / KT) : 0;
         ntiles = max(ntiles, ntl[t]);
     }
 
@@ -179,16 +188,16 @@ __global__ void __launch_bounds__(C::NT, 1)
         // holds entry win0 + l), refilled every 32/BPT tiles, so a tile's
         // copies are issued without a global round trip.
         constexpr int BPT = KT / 16;  // blocks per tile
-        int win0 = 0, went = bt[min(lane, nalloc - 1)];
+        int win0 = jt0 * BPT, went = bt[min(win0 + lane, nalloc - 1)];
         for (int j = 0; j < ntiles; ++j) {
-            const int s = j % NS;
+            const int s = j % NS, jb = (jt0 + j) * BPT;  // first block of the tile
             const uint32_t use = j / NS;  // how many times slot s was filled before
-            if (j * BPT + BPT > win0 + 32) {
-                win0 = j * BPT;
+            if (jb + BPT > win0 + 32) {
+                win0 = jb;
                 went = bt[min(win0 + lane, nalloc - 1)];
             }
-            // lanes 0..BPT-1: block j*BPT + lane (past the end: the last block, masked later)
-            int phys = __shfl_sync(0xffffffffu, went, (min(j * BPT + lane % BPT, nalloc - 1) - win0) & 31);
+            // lanes 0..BPT-1: block jb + lane (past the end: the last block, masked later)
+            int phys = __shfl_sync(0xffffffffu, went, (min(jb + lane % BPT, nalloc - 1) - win0) & 31);
             if (lane < BPT && (phys < 0 || phys >= a.num_blocks)) {
                 flag_error(a.err, PA_DEVERR_BAD_BLOCK);
                 phys = 0;
@@ -240,7 +249,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % NS, jn = j + 1, sn = jn % NS;
             ok = mbar_wait(&vfull[s], (j / NS) & 1) && ok;
-            const int kv0 = j * KT;
+            const int kv0 = (jt0 + j) * KT;
             if (kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
                 uint8_t *vt = sV + s * C::KTILE;
                 for (int r = max(L - kv0, 0) + lane; r < KT; r += 32)
@@ -321,7 +330,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             tmem_wait_ld();
             // raw scores (the scale is positive, so the max commutes with it);
             // the causal mask only where the tile reaches past this row
-            const int kv0 = j * KT + half * SCOL;
+            const int kv0 = (jt0 + j) * KT + half * SCOL;
             if (!(row_valid && kv0 + SCOL - 1 <= pos)) {
 #pragma unroll
                 for (int e = 0; e < SCOL; ++e) sv[e] = (row_valid && kv0 + e <= pos) ? sv[e] : -INFINITY;
@@ -381,7 +390,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             mbar_arrive(&pfull[t]);
         }
         if (ntl[t] > 0) {
-            // ---- epilogue: O / l, as bf16 output rows (or as split-K piece 0)
+            // ---- epilogue: O / l, as bf16 output rows (or as split-K piece kz)
             *xslot(2, half) = l;
             named_bar_sync(bar_id, 32 * NSP);
             l = 0.f;
@@ -393,9 +402,9 @@ __global__ void __launch_bounds__(C::NT, 1)
             __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;
             const float inv = (l > 0.f) ? 1.f / l : 0.f;
             if (shared) {
-                // split-K piece 0 of the row: normalised fp32 output and log2-sum-exp
+                // split-K piece kz of the row: normalised fp32 output and log2-sum-exp
                 const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;
-                float *wo = a.ws_o + grow * a.max_parts * D + half * OCOL;
+                float *wo = a.ws_o + (grow * a.max_parts + kz) * D + half * OCOL;
 #pragma unroll
                 for (int q = 0; q < OCOL / 32; ++q) {
                     float o[32];
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(C::NT, 1)
                                             o[e + 3] * inv * vs);
                     }
                 }
-                if (row_valid && half == 0) a.ws_lse[grow * a.max_parts] = (l > 0.f) ? m + lg2(l) : -INFINITY;
+                if (row_valid && half == 0) a.ws_lse[grow * a.max_parts + kz] = (l > 0.f) ? m + lg2(l) : -INFINITY;
             } else {
 #pragma unroll
                 for (int q = 0; q < OCOL / 32; ++q) {
@@ -490,7 +499,8 @@ cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
     CUtensorMap tk, tv;
     const int64_t rows = a.num_blocks * a.Hkv * 16;
     if (!cache_map(&tk, a.k_cache, rows, C::D) || !cache_map(&tv, a.v_cache, rows, C::D)) return cudaErrorInvalidValue;
-    dim3 grid((a.max_q_len + C::NQ * C::QPOS - 1) / (C::NQ * C::QPOS), a.Hkv, a.n_chunks);
+    dim3 grid((a.max_q_len + C::NQ * C::QPOS - 1) / (C::NQ * C::QPOS), a.Hkv,
+              a.shared_len > 0 ? std::max(a.key_splits, 1) : a.n_chunks);
     return launch_pdl(prefill_kernel<C>, grid, dim3(C::NT), C::SMEM, st, a, tk, tv);
 }
 

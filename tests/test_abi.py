@@ -104,3 +104,43 @@ def test_misaligned_pointers_are_rejected():
     d = desc()
     assert L.pa_write_kv(odd, FAKE, FAKE, 4, FAKE, FAKE, None, None, C.byref(d), None) == -1
     assert L.pa_copy_blocks(odd, FAKE, FAKE, 3, C.byref(d), None) == -1
+
+
+def call_cascade(d, B=4, maxb=8, Hq=32, pb=4, ws=FAKE, ws_bytes=1 << 30, ptr=FAKE, scales=FAKE):
+    return ops.lib().pa_decode_cascade(ptr, ptr, ptr, ptr, ptr, ptr, B, maxb, Hq, 0.1, scales, scales, pb, ws,
+                                       ws_bytes, C.byref(d) if d is not None else None, None)
+
+
+def test_cascade_rejects_bad_arguments_on_host():
+    assert call_cascade(None) == -1
+    assert call_cascade(desc(d=96)) == -2
+    assert call_cascade(desc(), pb=9) == -1          # more shared blocks than the table holds
+    assert call_cascade(desc(), pb=-1) == -1
+    assert call_cascade(desc(), Hq=30) == -1
+    assert call_cascade(desc(hkv=2), Hq=32) == -2    # group of 16 not built
+    assert call_cascade(desc(), B=5000) == -1
+    assert call_cascade(desc(), ptr=None) == -1
+    assert call_cascade(desc(dt=1), scales=None) == -1  # fp8 needs its scales
+    assert call_cascade(desc(), ws=None) == -3
+    assert call_cascade(desc(), ws_bytes=1024) == -3
+    assert call_cascade(desc(), ws=C.c_void_p(0x10010)) == -3  # not 256-byte aligned
+    assert call_cascade(desc(), B=0) == 0
+
+
+def cascade_ws(B, Hq, maxb, pb, dt=0, hkv=8, d=128):
+    out = C.c_size_t(0)
+    rc = ops.lib().pa_decode_cascade_workspace_size(B, Hq, maxb, pb, C.byref(desc(hkv=hkv, d=d, dt=dt)),
+                                                    C.byref(out))
+    return rc, out.value
+
+
+def test_cascade_workspace_size():
+    rc, n = cascade_ws(256, 64, 160, 128)
+    assert rc == 0
+    # split-K pieces of the 32-block suffix (at most 32/16 + 2) plus the prefix piece, fp32 o and lse
+    assert n >= 256 * 64 * 5 * (128 + 1) * 4
+    rc, n8 = cascade_ws(256, 64, 160, 128, dt=1)
+    assert rc == 0 and n8 >= n + 2 * 128 * 8 * 16 * 128 * 2  # fp8: the prefix widened to bf16
+    assert cascade_ws(256, 64, 160, 161)[0] == -1
+    assert cascade_ws(256, 64, 160, -1)[0] == -1
+    assert cascade_ws(256, 64, 160, 0)[1] >= ops.decode_workspace_size(256, 64, 128, 160)

@@ -274,3 +274,26 @@ def test_batch64_trace_keeps_64_sequences_and_utilisation_high():
     # replacements spend their admission step writing their prompt, then decode
     assert nd.max() <= 64 and nd.min() >= 56 and nd.mean() >= 62
     assert tr.sched.kv_utilisation() > 0.96  # paging wastes less than one block per sequence
+
+
+def test_shared_decode_blocks_is_the_common_fully_covered_table_prefix():
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        B, W = int(rng.integers(1, 6)), int(rng.integers(1, 9))
+        t = rng.integers(0, 3, (B, W)).astype(np.int32)
+        lens = rng.integers(1, 16 * W + 1, B).astype(np.int32)
+        plan = R.StepPlan(0, np.zeros((0, 2), np.int32), np.zeros(0, np.int64), np.arange(B), t, lens,
+                          np.zeros(0, np.int64), np.zeros(1, np.int32), np.zeros(0, np.int32),
+                          np.zeros((0, W), np.int32))
+        want = 0
+        while (want < W and all(t[b, want] == t[0, want] for b in range(B))
+               and all(lens[b] >= 16 * (want + 1) for b in range(B))):
+            want += 1
+        assert plan.shared_decode_blocks == want
+
+
+def test_forked_trace_shares_its_prompt_blocks_every_step():
+    from paged_kv_cache_408_b200 import traces
+    tr = traces.prefix_share_fp8(0, n=24, forks=4, prefix=256)
+    for plan in tr.plans(6):
+        assert plan.num_decode == 24 and plan.shared_decode_blocks >= 16
