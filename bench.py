@@ -150,6 +150,12 @@ def decode_alg_flops(lens, Hq, D):
     return 4 * D * Hq * int(np.asarray(lens, np.int64).sum())
 
 
+def decode_math_on_cuda_cores(Hq, Hkv, fp8):
+    """The decode kernel does q.k and p.v on the CUDA cores except for an fp8
+    cache with GQA 8, where it uses the tensor cores (mma.sync, f16)."""
+    return not (fp8 and Hq // Hkv == 8)
+
+
 def alu_peak(sm_mhz):
     """fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per
     clock, at the SM clock sampled during the timed region."""
@@ -645,7 +651,7 @@ def aggregate(tot_s, kv_bytes_done, seq_steps, world, device):
 
 
 
-def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload):
+def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload, cuda_core_math=True):
     """Roofline of a cascade decode call (fp8 widening, prefix attention on
     the tensor cores, suffix decode, merge).  The suffix stage is timed on
     its own (the decode kernel over the suffix tables); the prefix stage is
@@ -659,7 +665,8 @@ def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload):
               "peak_kind": tkind, "kernel": "prefill_kernel (shared-prefix mode) + fp8 widening",
               "ms_per_launch": t_pre * 1e3, "alg_flops_per_launch": c["prefix_flops"],
               "timing": "cascade call minus the suffix stage timed alone", "traffic": None}
-    if c["suffix_flops"] / (apeak * 1e12) > c["suffix_bytes"] / (hbm_peak * 1e9):
+    alu_s = c["suffix_flops"] / (apeak * 1e12) if cuda_core_math else c["suffix_flops"] / (tpeak * 1e12)
+    if cuda_core_math and alu_s > c["suffix_bytes"] / (hbm_peak * 1e9):
         tfl = c["suffix_flops"] / t_sfx / 1e12
         suffix = {"bound": "alu", "achieved": tfl, "peak": apeak, "unit": "TFLOP/s", "frac": tfl / apeak,
                   "peak_kind": f"derived: 148 SMs x 128 fp32 lanes x 2 FLOP x {sm_mhz:.0f} MHz"}
@@ -672,7 +679,7 @@ def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload):
                    "timing": "decode call over the suffix tables, CUDA events",
                    "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", workload + ":suffix")})
     roof_s = (c["prefix_flops"] / (tpeak * 1e12) +
-              max(c["suffix_flops"] / (apeak * 1e12), c["suffix_bytes"] / (hbm_peak * 1e9)))
+              max(alu_s, c["suffix_bytes"] / (hbm_peak * 1e9)))
     out = dict(suffix if t_sfx >= t_pre else prefix)
     out["stages"] = {"prefix": prefix, "suffix": suffix,
                      "call": {"ms_per_launch": t_call * 1e3, "roof_ms": roof_s * 1e3, "frac": roof_s / t_call,
@@ -735,11 +742,12 @@ def main():
         alg = sum(r["algb"]) / len(r["algb"])
         flops = sum(r["algf"]) / len(r["algf"])
         achieved = alg / (dec_ms / 1e3) / 1e9
-        # the binding roof: HBM bytes or CUDA-core FLOPs (GQA 8 with an fp8
-        # cache does 16 FLOP per cached byte and is arithmetic-bound)
+        # the binding roof: HBM bytes, or CUDA-core FLOPs where the decode
+        # kernel does its products on the CUDA cores and they take longer
         sm_mhz = (r["clocks"] or {}).get("sm_mhz") or 1965.0
         apeak = alu_peak(sm_mhz)
-        alu_bound = flops / (apeak * 1e12) > alg / (peak * 1e9)
+        cuda_core_math = decode_math_on_cuda_cores(r.get("Hq", 32), r.get("Hkv", 8), r["fp8"])
+        alu_bound = cuda_core_math and flops / (apeak * 1e12) > alg / (peak * 1e9)
         if alu_bound:
             tfl = flops / (dec_ms / 1e3) / 1e12
             roof = {"bound": "alu", "achieved": tfl, "peak": apeak, "unit": "TFLOP/s", "frac": tfl / apeak,
@@ -752,7 +760,7 @@ def main():
                      "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", args.workload),
                      "alg_bytes_per_launch": alg, "alg_flops_per_launch": flops, "ms_per_launch": dec_ms})
         if r.get("cascade"):
-            roof = cascade_roofline(r["cascade"], peak, peak_kind, apeak, sm_mhz, args.workload)
+            roof = cascade_roofline(r["cascade"], peak, peak_kind, apeak, sm_mhz, args.workload, cuda_core_math)
         tr = r["tr"]
         line = {
             "metric": METRIC, "value": kvb / tot_s / 1e9, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

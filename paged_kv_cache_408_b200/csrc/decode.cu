@@ -38,8 +38,11 @@
 //    SM's warps fill kRingBytes of shared memory.  The producer runs ahead
 //    across item boundaries and keeps block-table entries in registers (a
 //    sliding window, plus the next item's first entries).
-//  * Math on CUDA cores (4-8 query rows per step are far below a
-//    tensor-core tile): lanes form token groups of LPT lanes; a lane owns
+//  * Math on CUDA cores for bf16 caches and for groups of up to 4 heads
+//    (4-8 query rows are far below a tcgen05 tile, and the path is
+//    HBM-bound), on the tensor cores with warp-level MMAs for an fp8 cache
+//    with groups of 8 (see mma_items).  CUDA-core path: lanes form token
+//    groups of LPT lanes; a lane owns
 //    DPL head dims (16-byte shared-memory reads, bank-conflict-free), keeps
 //    q for them in fp32 registers pre-scaled by scale*log2(e), and
 //    accumulates with packed fp32x2 FMAs.  Partial dot products are
@@ -93,8 +96,10 @@ struct Cfg {
     // CTAS CTAs of NW warps per SM share the register file (G = 8 needs ~255
     // registers a thread, so 8 warps an SM; otherwise ~168, so 12) and a
     // kRingBytes shared-memory ring, split into NSTAGE stages per warp.
-    static constexpr int CTAS = (G >= 8) ? 2 : 1;     // CTAs per SM
-    static constexpr int NW = (G >= 8) ? 4 : 12;      // warps per CTA
+    // fp8 with GQA 8 runs its products on the tensor cores (mma_items)
+    static constexpr bool MMA = FP8 && G == 8;
+    static constexpr int CTAS = (G >= 8 && !MMA) ? 2 : 1;  // CTAs per SM
+    static constexpr int NW = (G >= 8 && !MMA) ? 4 : 12;   // warps per CTA
     static constexpr int NT = NW * 32;
     static constexpr int NSTAGE = (int)(kRingBytes / ((size_t)CTAS * NW * 2 * BLKB));  // ring depth per warp
     static constexpr int MIN_CTAS = CTAS;
@@ -418,6 +423,272 @@ struct QPrefetch {
     }
 };
 
+// ---- tensor-core decode (fp8 cache, GQA groups of 8) ----------------------
+//
+// With an fp8 cache and 8 q heads per kv head, q.k and p.v on CUDA cores
+// cost 16 FLOP per cached byte, more than the fp32 pipes deliver at HBM
+// speed.  This path moves both products onto the tensor cores with the
+// warp-level mma.sync m16n8k16 (f16 operands, fp32 accumulators), one block
+// (16 tokens) at a time:
+//     S^T [16 tokens x 8 heads]  = K [16 x D] . q^T [D x 8]      (D/16 MMAs)
+//     O^T [D x 8 heads]         += V^T [D x 16] . P^T [16 x 8]   (D/16 MMAs)
+// so no operand is padded.  E4M3 codes widen to f16 exactly; q is scaled
+// by a power of two 2^e so that its largest magnitude lies in [2^14, 2^15)
+// (exact for every bf16 value in f16's normal range; 2^-e is folded into
+// the softmax scale).  P is rounded to f16 for the MMA (the normaliser
+// sums the fp32 values).
+//
+// Index maps (a reduction index may be permuted freely as long as both
+// operands use the same map): lane (r = lane/4, c = lane%4) reads, of K,
+// rows r and r+8 at dims [c*D/4, (c+1)*D/4), so its k-indices
+// {2c, 2c+1, 2c+8, 2c+9} of MMA step kk are dims c*D/4 + 4kk + {0,1,2,3}:
+// one 32-bit shared-memory word per row and step; q uses the same map.  Of
+// V it reads tokens {2c, 2c+1, 2c+8, 2c+9} at dims [r*D/8, (r+1)*D/8): row
+// m = r of output tile mt is dim r*D/8 + mt, row r+8 is r*D/8 + D/16 + mt,
+// so the lane's output for one head is D/8 contiguous dims.  The S^T
+// accumulator tile, transposed by movmatrix, is exactly P^T's B fragment.
+PA_DEVICE void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+PA_DEVICE uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Two E4M3 codes (low byte first) -> f16x2, exact.
+PA_DEVICE uint32_t e4m3x2_to_h2(uint32_t w16) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w16 & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+PA_DEVICE uint32_t f2_to_h2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+PA_DEVICE uint32_t prmt(uint32_t x, uint32_t y, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(x), "r"(y), "r"(sel));
+    return d;
+}
+
+// q of one item for the tensor-core path: head r, dims [c*D/4, (c+1)*D/4).
+template <class C>
+struct QPrefetchMma {
+    static constexpr int NQ4 = C::D / 32;  // uint4 (8 bf16) per lane
+    uint4 q[NQ4];
+    float ks, vs;
+
+    PA_DEVICE void load(const DecodeArgs &a, const Item &it, int r, int c) {
+        const __nv_bfloat16 *qrow = static_cast<const __nv_bfloat16 *>(a.q) +
+                                    ((size_t)it.b * a.Hq + (size_t)it.kvh * C::G + r) * C::D + c * (C::D / 4);
+#pragma unroll
+        for (int i = 0; i < NQ4; ++i) q[i] = reinterpret_cast<const uint4 *>(qrow)[i];
+        ks = a.k_scale[it.kvh];
+        vs = a.v_scale[it.kvh];
+    }
+};
+
+template <class C>
+PA_DEVICE void mma_items(const DecodeArgs &a, const Schedule &sc, Producer<C> &prod, ItemIter &items,
+                         uint8_t *my_stages, uint64_t *my_bars, int *my_valid, int lane, const uint8_t *kc,
+                         const uint8_t *vc) {
+    constexpr int D = C::D, G = C::G, NK = D / 16, NM = D / 16, KW = D / 16, VB = D / 8;
+    static_assert(C::FP8 && G == 8, "tensor-core decode: fp8 cache, GQA 8");
+    const int r = lane >> 2, c = lane & 3, Hkv = sc.Hkv;
+    uint32_t consumed = 0;
+    Item it, nx;
+    bool have = items.next(sc, it);
+    bool have_nx = have && items.next(sc, nx);
+    QPrefetchMma<C> qp;
+    if (have) qp.load(a, it, r, c);
+    while (have) {
+        const float vscale = qp.vs;
+        // ---- q^T fragments in f16 with a power-of-two scale 2^e
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < QPrefetchMma<C>::NQ4; ++i) {
+            const uint32_t ws[4] = {qp.q[i].x, qp.q[i].y, qp.q[i].z, qp.q[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = bf16x2_to_float2(ws[e]);
+                amax = fmax3(amax, fabsf(f.x), fabsf(f.y));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, o));
+        int ex = 0;
+        if (amax > 0.f) ex = min(max(14 - ((int)((__float_as_uint(amax) >> 23) & 0xff) - 127), -60), 60);
+        const float qsc = __uint_as_float((uint32_t)(127 + ex) << 23);
+        const float sl2 = a.scale * kLog2e * qp.ks * __uint_as_float((uint32_t)(127 - ex) << 23);
+        uint32_t qf[NK][2];
+#pragma unroll
+        for (int kk = 0; kk < NK; ++kk) {
+            const uint4 u = qp.q[kk / 2];
+            const uint32_t w0 = (kk & 1) ? u.z : u.x, w1 = (kk & 1) ? u.w : u.y;
+            const float2 f0 = bf16x2_to_float2(w0), f1 = bf16x2_to_float2(w1);
+            qf[kk][0] = f2_to_h2(f0.x * qsc, f0.y * qsc);
+            qf[kk][1] = f2_to_h2(f1.x * qsc, f1.y * qsc);
+        }
+        float o[NM][4];
+#pragma unroll
+        for (int mt = 0; mt < NM; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2c, 2c+1
+
+        for (int j = 0; j < it.nblk; ++j) {
+            const int s = consumed % C::NSTAGE;
+            if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
+                flag_error(a.err, PA_DEVERR_TIMEOUT);
+            const int valid = my_valid[s];
+            const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
+            // ---- S^T = K q^T
+            uint32_t kr[KW], kr8[KW];
+#pragma unroll
+            for (int i = 0; i < KW / 4; ++i) {
+                const uint4 u = *reinterpret_cast<const uint4 *>(Kb + r * D + c * (D / 4) + 16 * i);
+                const uint4 u8 = *reinterpret_cast<const uint4 *>(Kb + (r + 8) * D + c * (D / 4) + 16 * i);
+                kr[4 * i] = u.x, kr[4 * i + 1] = u.y, kr[4 * i + 2] = u.z, kr[4 * i + 3] = u.w;
+                kr8[4 * i] = u8.x, kr8[4 * i + 1] = u8.y, kr8[4 * i + 2] = u8.z, kr8[4 * i + 3] = u8.w;
+            }
+            float st[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < NK; ++kk)
+                mma_f16(st, e4m3x2_to_h2(kr[kk]), e4m3x2_to_h2(kr8[kk]), e4m3x2_to_h2(kr[kk] >> 16),
+                        e4m3x2_to_h2(kr8[kk] >> 16), qf[kk][0], qf[kk][1]);
+            // V rows of this lane's tokens, loaded now so they overlap the softmax
+            uint32_t vw[4][VB / 4];
+            {
+                const int tok[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint8_t *src = Vb + tok[t] * D + r * VB;
+                    if constexpr (VB == 16) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(src);
+                        vw[t][0] = u.x, vw[t][1] = u.y, vw[t][2] = u.z, vw[t][3] = u.w;
+                    } else {
+                        const uint2 u = *reinterpret_cast<const uint2 *>(src);
+                        vw[t][0] = u.x, vw[t][1] = u.y;
+                    }
+                }
+                if (valid < 16) {  // rows past the end may hold any bytes (NaN codes): zero them
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        if (tok[t] >= valid)
+#pragma unroll
+                            for (int i = 0; i < VB / 4; ++i) vw[t][i] = 0u;
+                }
+            }
+            // ---- online softmax over the block's tokens, heads 2c and 2c+1
+            const bool ok0 = r < valid, ok8 = r + 8 < valid;
+            const float t0 = ok0 ? st[0] * sl2 : -INFINITY, t1 = ok0 ? st[1] * sl2 : -INFINITY;
+            const float t2 = ok8 ? st[2] * sl2 : -INFINITY, t3 = ok8 ? st[3] * sl2 : -INFINITY;
+            const bool need = fmaxf(t0, t2) > m0 + kRescaleThreshold || fmaxf(t1, t3) > m1 + kRescaleThreshold;
+            if (__any_sync(kFull, need)) {
+                float b0 = fmaxf(t0, t2), b1 = fmaxf(t1, t3);
+#pragma unroll
+                for (int x = 4; x <= 16; x <<= 1) {
+                    b0 = fmaxf(b0, __shfl_xor_sync(kFull, b0, x));
+                    b1 = fmaxf(b1, __shfl_xor_sync(kFull, b1, x));
+                }
+                const float n0 = fmaxf(m0, b0), n1 = fmaxf(m1, b1);
+                const float al0 = (n0 == -INFINITY) ? 1.f : ex2(m0 - n0), al1 = (n1 == -INFINITY) ? 1.f : ex2(m1 - n1);
+                m0 = n0, m1 = n1;
+                l0 *= al0, l1 *= al1;
+#pragma unroll
+                for (int mt = 0; mt < NM; ++mt) {
+                    o[mt][0] *= al0, o[mt][2] *= al0;
+                    o[mt][1] *= al1, o[mt][3] *= al1;
+                }
+            }
+            const float mb0 = (m0 == -INFINITY) ? 0.f : m0, mb1 = (m1 == -INFINITY) ? 0.f : m1;
+            const float p0 = ex2(t0 - mb0), p1 = ex2(t1 - mb1), p2 = ex2(t2 - mb0), p3 = ex2(t3 - mb1);
+            l0 += p0 + p2;
+            l1 += p1 + p3;
+            // P^T fragments: the accumulator tile (tokens x heads) transposed
+            const uint32_t pb0 = movmatrix_trans(f2_to_h2(p0, p1)), pb1 = movmatrix_trans(f2_to_h2(p2, p3));
+            // ---- O^T += V^T P^T, two output tiles per byte-pair permute
+#pragma unroll
+            for (int mt = 0; mt < NM; mt += 2) {
+                const int w = mt / 4, bsel = mt % 4;
+                const uint32_t sel = bsel | ((4 + bsel) << 4) | ((bsel + 1) << 8) | ((5 + bsel) << 12);
+                constexpr int HW = (D / 16) / 4;  // word offset of the rows r+8 dims
+                const uint32_t x0 = prmt(vw[0][w], vw[1][w], sel);            // tokens 2c, 2c+1, row r
+                const uint32_t x1 = prmt(vw[0][w + HW], vw[1][w + HW], sel);  // tokens 2c, 2c+1, row r+8
+                const uint32_t x2 = prmt(vw[2][w], vw[3][w], sel);            // tokens 2c+8, 2c+9, row r
+                const uint32_t x3 = prmt(vw[2][w + HW], vw[3][w + HW], sel);
+                mma_f16(o[mt], e4m3x2_to_h2(x0), e4m3x2_to_h2(x1), e4m3x2_to_h2(x2), e4m3x2_to_h2(x3), pb0, pb1);
+                mma_f16(o[mt + 1], e4m3x2_to_h2(x0 >> 16), e4m3x2_to_h2(x1 >> 16), e4m3x2_to_h2(x2 >> 16),
+                        e4m3x2_to_h2(x3 >> 16), pb0, pb1);
+            }
+            __syncwarp();
+            ++consumed;
+            prod.produce(sc, a, lane, kc, vc, my_stages, my_bars, my_valid);
+        }
+        if (have_nx) qp.load(a, nx, r, c);
+
+        // ---- epilogue: the normalisers over the lanes of each head
+#pragma unroll
+        for (int x = 4; x <= 16; x <<= 1) {
+            l0 += __shfl_xor_sync(kFull, l0, x);
+            l1 += __shfl_xor_sync(kFull, l1, x);
+        }
+        const size_t row0 = (size_t)it.b * a.Hq + (size_t)it.kvh * G;
+        const float inv0 = (l0 > 0.f) ? vscale / l0 : 0.f, inv1 = (l1 > 0.f) ? vscale / l1 : 0.f;
+        // head 2c: o[.][0] (dims r*VB + mt) then o[.][2] (dims r*VB + NM + mt); head 2c+1: [1], [3]
+        if (it.npieces == 1 && !a.prefix_blocks) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const float inv = hh ? inv1 : inv0;
+                uint32_t wds[VB / 2];
+#pragma unroll
+                for (int i = 0; i < VB / 2; ++i) {
+                    const int d0 = 2 * i, d1 = 2 * i + 1;  // dims r*VB + d
+                    const float v0 = d0 < NM ? o[d0][hh] : o[d0 - NM][2 + hh];
+                    const float v1 = d1 < NM ? o[d1][hh] : o[d1 - NM][2 + hh];
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(v0 * inv, v1 * inv);
+                    wds[i] = *reinterpret_cast<const uint32_t *>(&bb);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) +
+                                                       (row0 + 2 * c + hh) * D + r * VB);
+#pragma unroll
+                for (int i = 0; i < VB / 8; ++i) dst[i] = make_uint4(wds[4 * i], wds[4 * i + 1], wds[4 * i + 2], wds[4 * i + 3]);
+            }
+            if (lane == 0 && a.ws_np) a.ws_np[(size_t)it.b * Hkv + it.kvh] = 1;
+        } else {
+            const int piece = it.piece + a.prefix_pieces;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const float inv = hh ? inv1 : inv0;
+                float4 *dst = reinterpret_cast<float4 *>(a.ws_o + ((row0 + 2 * c + hh) * a.max_parts + piece) * D + r * VB);
+#pragma unroll
+                for (int i = 0; i < VB / 4; ++i) {
+                    float v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int d = 4 * i + e;
+                        v[e] = (d < NM ? o[d][hh] : o[d - NM][2 + hh]) * inv;
+                    }
+                    dst[i] = make_float4(v[0], v[1], v[2], v[3]);
+                }
+            }
+            if (r == 0) {
+                a.ws_lse[(row0 + 2 * c) * a.max_parts + piece] = (l0 > 0.f) ? m0 + lg2(l0) : -INFINITY;
+                a.ws_lse[(row0 + 2 * c + 1) * a.max_parts + piece] = (l1 > 0.f) ? m1 + lg2(l1) : -INFINITY;
+            }
+            if (lane == 0 && it.piece == 0) a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces + a.prefix_pieces;
+        }
+        it = nx;
+        have = have_nx;
+        have_nx = have && items.next(sc, nx);
+    }
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const DecodeArgs a) {
     constexpr int D = C::D, G = C::G, NW = C::NW, NS = C::NS, VPL = C::VPL, P2 = C::P2, LPT = C::LPT;
@@ -548,181 +819,185 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
 
     ItemIter items;
     items.start(sc, gw, GW);
-    Item it, nx;
-    bool have = items.next(sc, it);
-    bool have_nx = have && items.next(sc, nx);
-    QPrefetch<C> qp;
-    if (have) qp.load(a, it, choff, sh);
-    while (have) {
-        const float vscale = qp.vs;
-        const float qs = a.scale * kLog2e * qp.ks;
-        const size_t row0 = (size_t)it.b * a.Hq + (size_t)it.kvh * G;  // first q head of the group
+    if constexpr (C::MMA) {
+        mma_items<C>(a, sc, prod, items, my_stages, my_bars, my_valid, lane, kc, vc);
+    } else {
+        Item it, nx;
+        bool have = items.next(sc, it);
+        bool have_nx = have && items.next(sc, nx);
+        QPrefetch<C> qp;
+        if (have) qp.load(a, it, choff, sh);
+        while (have) {
+            const float vscale = qp.vs;
+            const float qs = a.scale * kLog2e * qp.ks;
+            const size_t row0 = (size_t)it.b * a.Hq + (size_t)it.kvh * G;  // first q head of the group
 
-        // q of the GQA group in fp32, pre-scaled into log2 units; slot h = head h ^ sh
-        float2 q2[G][P2], acc2[G][P2];
-        float m[G], l[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-#pragma unroll
-            for (int c = 0; c < C::NCH; ++c) {
-                const uint32_t ws[4] = {qp.q[h][c].x, qp.q[h][c].y, qp.q[h][c].z, qp.q[h][c].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = bf16x2_to_float2(ws[e]);
-                    q2[h][4 * c + e] = make_float2(f.x * qs, f.y * qs);
-                    acc2[h][4 * c + e] = make_float2(0.f, 0.f);
+            // q of the GQA group in fp32, pre-scaled into log2 units; slot h = head h ^ sh
+            float2 q2[G][P2], acc2[G][P2];
+            float m[G], l[G];
+    #pragma unroll
+            for (int h = 0; h < G; ++h) {
+    #pragma unroll
+                for (int c = 0; c < C::NCH; ++c) {
+                    const uint32_t ws[4] = {qp.q[h][c].x, qp.q[h][c].y, qp.q[h][c].z, qp.q[h][c].w};
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = bf16x2_to_float2(ws[e]);
+                        q2[h][4 * c + e] = make_float2(f.x * qs, f.y * qs);
+                        acc2[h][4 * c + e] = make_float2(0.f, 0.f);
+                    }
                 }
+                m[h] = -INFINITY;
+                l[h] = 0.f;
             }
-            m[h] = -INFINITY;
-            l[h] = 0.f;
-        }
 
-        for (int j = 0; j < it.nblk; ++j) {
-            const int s = consumed % C::NSTAGE;
-            if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
-                flag_error(a.err, PA_DEVERR_TIMEOUT);
-            const int valid = my_valid[s];
-            const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
+            for (int j = 0; j < it.nblk; ++j) {
+                const int s = consumed % C::NSTAGE;
+                if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
+                    flag_error(a.err, PA_DEVERR_TIMEOUT);
+                const int valid = my_valid[s];
+                const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
 
-#pragma unroll
-            for (int sb = 0; sb < C::NSUB; ++sb) {
-                const int t_base = g + C::NGRP * sb * C::TSUB;
-                // --- q . k: partial dot products over this lane's dims
-                float part[NS];
-#pragma unroll
-                for (int jj = 0; jj < C::TSUB; ++jj) {
-                    float2 kf[P2];
-                    load_row<C>(Kb + (t_base + C::NGRP * (jj ^ sj)) * C::ROWB, choff, kf);
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        float2 d2 = make_float2(0.f, 0.f);
-#pragma unroll
-                        for (int k = 0; k < P2; ++k) d2 = ffma2(q2[h][k], kf[k], d2);
-                        part[jj * G + h] = d2.x + d2.y;
-                    }
-                }
-                // --- complete the scores across the LPT lanes of the group
-                if constexpr (C::RS)
-                    rs_level<LPT / 2, NS / 2, NS>(part);
-                else
-                    allreduce_level<LPT / 2, NS>(part);
-                // --- owned score i: head slot i % G, token slot i / G.
-                // Mask tokens past the end; move the running max only when a
-                // score exceeds it by more than the threshold.
-                float sco[VPL];
-                bool need = false;
-#pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int t = t_base + C::NGRP * ((i / G) ^ sj);
-                    sco[i] = (t < valid) ? part[i] : -INFINITY;
-                    need |= sco[i] > m[i % G] + kRescaleThreshold;
-                }
-                if (__any_sync(kFull, need)) {
-                    float bm[G];
-#pragma unroll
-                    for (int h = 0; h < G; ++h) bm[h] = -INFINITY;
-#pragma unroll
-                    for (int i = 0; i < VPL; ++i) bm[i % G] = fmaxf(bm[i % G], sco[i]);
-                    if constexpr (C::RS) perm_allreduce<LPT / 2, VPL, G, true>(bm);
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float mn = fmaxf(m[h], bm[h]);
-                        const float alpha = (mn == -INFINITY) ? 1.f : ex2(m[h] - mn);
-                        m[h] = mn;
-                        l[h] *= alpha;
-#pragma unroll
-                        for (int k = 0; k < P2; ++k) acc2[h][k] = fmul2(acc2[h][k], make_float2(alpha, alpha));
-                    }
-                }
-                // --- probabilities of the owned scores, then all-gather them
-                float pr[NS];
-#pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const float p = (sco[i] == -INFINITY) ? 0.f : ex2(sco[i] - m[i % G]);
-                    l[i % G] += p;
-                    pr[i] = p;
-                }
-                if constexpr (C::RS) ag_level<1, LPT, VPL, NS>(pr);
-                // --- acc += p * v over this group's tokens
-#pragma unroll
-                for (int jj = 0; jj < C::TSUB; ++jj) {
-                    const int t = t_base + C::NGRP * (jj ^ sj);
-                    if (t < valid) {
-                        float2 vf[P2];
-                        load_row<C>(Vb + t * C::ROWB, choff, vf);
-#pragma unroll
+    #pragma unroll
+                for (int sb = 0; sb < C::NSUB; ++sb) {
+                    const int t_base = g + C::NGRP * sb * C::TSUB;
+                    // --- q . k: partial dot products over this lane's dims
+                    float part[NS];
+    #pragma unroll
+                    for (int jj = 0; jj < C::TSUB; ++jj) {
+                        float2 kf[P2];
+                        load_row<C>(Kb + (t_base + C::NGRP * (jj ^ sj)) * C::ROWB, choff, kf);
+    #pragma unroll
                         for (int h = 0; h < G; ++h) {
-                            const float p = pr[jj * G + h];
-                            const float2 pp = make_float2(p, p);
-#pragma unroll
-                            for (int k = 0; k < P2; ++k) acc2[h][k] = ffma2(pp, vf[k], acc2[h][k]);
+                            float2 d2 = make_float2(0.f, 0.f);
+    #pragma unroll
+                            for (int k = 0; k < P2; ++k) d2 = ffma2(q2[h][k], kf[k], d2);
+                            part[jj * G + h] = d2.x + d2.y;
+                        }
+                    }
+                    // --- complete the scores across the LPT lanes of the group
+                    if constexpr (C::RS)
+                        rs_level<LPT / 2, NS / 2, NS>(part);
+                    else
+                        allreduce_level<LPT / 2, NS>(part);
+                    // --- owned score i: head slot i % G, token slot i / G.
+                    // Mask tokens past the end; move the running max only when a
+                    // score exceeds it by more than the threshold.
+                    float sco[VPL];
+                    bool need = false;
+    #pragma unroll
+                    for (int i = 0; i < VPL; ++i) {
+                        const int t = t_base + C::NGRP * ((i / G) ^ sj);
+                        sco[i] = (t < valid) ? part[i] : -INFINITY;
+                        need |= sco[i] > m[i % G] + kRescaleThreshold;
+                    }
+                    if (__any_sync(kFull, need)) {
+                        float bm[G];
+    #pragma unroll
+                        for (int h = 0; h < G; ++h) bm[h] = -INFINITY;
+    #pragma unroll
+                        for (int i = 0; i < VPL; ++i) bm[i % G] = fmaxf(bm[i % G], sco[i]);
+                        if constexpr (C::RS) perm_allreduce<LPT / 2, VPL, G, true>(bm);
+    #pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float mn = fmaxf(m[h], bm[h]);
+                            const float alpha = (mn == -INFINITY) ? 1.f : ex2(m[h] - mn);
+                            m[h] = mn;
+                            l[h] *= alpha;
+    #pragma unroll
+                            for (int k = 0; k < P2; ++k) acc2[h][k] = fmul2(acc2[h][k], make_float2(alpha, alpha));
+                        }
+                    }
+                    // --- probabilities of the owned scores, then all-gather them
+                    float pr[NS];
+    #pragma unroll
+                    for (int i = 0; i < VPL; ++i) {
+                        const float p = (sco[i] == -INFINITY) ? 0.f : ex2(sco[i] - m[i % G]);
+                        l[i % G] += p;
+                        pr[i] = p;
+                    }
+                    if constexpr (C::RS) ag_level<1, LPT, VPL, NS>(pr);
+                    // --- acc += p * v over this group's tokens
+    #pragma unroll
+                    for (int jj = 0; jj < C::TSUB; ++jj) {
+                        const int t = t_base + C::NGRP * (jj ^ sj);
+                        if (t < valid) {
+                            float2 vf[P2];
+                            load_row<C>(Vb + t * C::ROWB, choff, vf);
+    #pragma unroll
+                            for (int h = 0; h < G; ++h) {
+                                const float p = pr[jj * G + h];
+                                const float2 pp = make_float2(p, p);
+    #pragma unroll
+                                for (int k = 0; k < P2; ++k) acc2[h][k] = ffma2(pp, vf[k], acc2[h][k]);
+                            }
                         }
                     }
                 }
+                __syncwarp();
+                ++consumed;
+                prod.produce(sc, a, lane, kc, vc, my_stages, my_bars, my_valid);
             }
-            __syncwarp();
-            ++consumed;
-            prod.produce(sc, a, lane, kc, vc, my_stages, my_bars, my_valid);
-        }
 
-        // ---- the next item's q and scales are needed right after this
-        // epilogue: start their loads now so the latency overlaps it
-        if (have_nx) qp.load(a, nx, choff, sh);
+            // ---- the next item's q and scales are needed right after this
+            // epilogue: start their loads now so the latency overlaps it
+            if (have_nx) qp.load(a, nx, choff, sh);
 
-        // ---- epilogue: complete the normaliser per head across the group,
-        // then merge the token groups (same dims, different tokens)
-        if constexpr (C::RS) perm_allreduce<LPT / 2, VPL, G, false>(l);
-        group_merge<LPT, LPT, G, P2, C::NCH == 2>(m, l, acc2);
+            // ---- epilogue: complete the normaliser per head across the group,
+            // then merge the token groups (same dims, different tokens)
+            if constexpr (C::RS) perm_allreduce<LPT / 2, VPL, G, false>(l);
+            group_merge<LPT, LPT, G, P2, C::NCH == 2>(m, l, acc2);
 
-        // every group now holds the warp's result; group 0 writes it
-        if (it.npieces == 1 && !a.prefix_blocks) {
-            if (g == 0) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + (row0 + (h ^ sh)) * D;
-#pragma unroll
-                    for (int c = 0; c < C::NCH; ++c) {
-                        uint32_t wds[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 bb =
-                                __floats2bfloat162_rn(acc2[h][4 * c + e].x * inv, acc2[h][4 * c + e].y * inv);
-                            wds[e] = *reinterpret_cast<const uint32_t *>(&bb);
+            // every group now holds the warp's result; group 0 writes it
+            if (it.npieces == 1 && !a.prefix_blocks) {
+                if (g == 0) {
+    #pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
+                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + (row0 + (h ^ sh)) * D;
+    #pragma unroll
+                        for (int c = 0; c < C::NCH; ++c) {
+                            uint32_t wds[4];
+    #pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 bb =
+                                    __floats2bfloat162_rn(acc2[h][4 * c + e].x * inv, acc2[h][4 * c + e].y * inv);
+                                wds[e] = *reinterpret_cast<const uint32_t *>(&bb);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + choff[c] * 8) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
                         }
-                        *reinterpret_cast<uint4 *>(dst + choff[c] * 8) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
                     }
                 }
-            }
-            if (lane == 0 && a.ws_np) a.ws_np[(size_t)it.b * Hkv + it.kvh] = 1;  // nothing to merge
-        } else {
-            // ---- split-K: this piece's normalised output and log2-sum-exp;
-            // piece 0 also records how many pieces the merge kernel combines
-            // (in a cascade the pieces follow the shared prefix's pieces)
-            const int piece = it.piece + a.prefix_pieces;
-            if (g == 0) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
-                    float *dst = a.ws_o + ((row0 + (h ^ sh)) * a.max_parts + piece) * D;
-#pragma unroll
-                    for (int c = 0; c < C::NCH; ++c) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + choff[c] * 8);
-                        d4[0] = make_float4(acc2[h][4 * c].x * inv, acc2[h][4 * c].y * inv,
-                                            acc2[h][4 * c + 1].x * inv, acc2[h][4 * c + 1].y * inv);
-                        d4[1] = make_float4(acc2[h][4 * c + 2].x * inv, acc2[h][4 * c + 2].y * inv,
-                                            acc2[h][4 * c + 3].x * inv, acc2[h][4 * c + 3].y * inv);
+                if (lane == 0 && a.ws_np) a.ws_np[(size_t)it.b * Hkv + it.kvh] = 1;  // nothing to merge
+            } else {
+                // ---- split-K: this piece's normalised output and log2-sum-exp;
+                // piece 0 also records how many pieces the merge kernel combines
+                // (in a cascade the pieces follow the shared prefix's pieces)
+                const int piece = it.piece + a.prefix_pieces;
+                if (g == 0) {
+    #pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float inv = (l[h] > 0.f) ? vscale / l[h] : 0.f;
+                        float *dst = a.ws_o + ((row0 + (h ^ sh)) * a.max_parts + piece) * D;
+    #pragma unroll
+                        for (int c = 0; c < C::NCH; ++c) {
+                            float4 *d4 = reinterpret_cast<float4 *>(dst + choff[c] * 8);
+                            d4[0] = make_float4(acc2[h][4 * c].x * inv, acc2[h][4 * c].y * inv,
+                                                acc2[h][4 * c + 1].x * inv, acc2[h][4 * c + 1].y * inv);
+                            d4[1] = make_float4(acc2[h][4 * c + 2].x * inv, acc2[h][4 * c + 2].y * inv,
+                                                acc2[h][4 * c + 3].x * inv, acc2[h][4 * c + 3].y * inv);
+                        }
+                        if (sub == 0)  // sub 0 has sh == 0: slot h is head h
+                            a.ws_lse[(row0 + h) * a.max_parts + piece] = (l[h] > 0.f) ? m[h] + lg2(l[h]) : -INFINITY;
                     }
-                    if (sub == 0)  // sub 0 has sh == 0: slot h is head h
-                        a.ws_lse[(row0 + h) * a.max_parts + piece] = (l[h] > 0.f) ? m[h] + lg2(l[h]) : -INFINITY;
                 }
+                if (lane == 0 && it.piece == 0)
+                    a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces + a.prefix_pieces;
             }
-            if (lane == 0 && it.piece == 0)
-                a.ws_np[(size_t)it.b * Hkv + it.kvh] = it.npieces + a.prefix_pieces;
+            it = nx;
+            have = have_nx;
+            have_nx = have && items.next(sc, nx);
         }
-        it = nx;
-        have = have_nx;
-        have_nx = have && items.next(sc, nx);
     }
 }
 
