@@ -1131,8 +1131,9 @@ cudaError_t run(const DecodeArgs &a, cudaStream_t st) {
         ctas = slot->ctas * sms[dev];
     }
     // enough CTAs to cover every warp-sized unit of work, at most one wave
+    // (balanced: a segment costs its blocks plus kSegmentCost units)
     const long long units = a.partition_tokens == 0
-                                ? (long long)a.Hkv * a.B * a.max_blocks / kMinShareBlocks + 1
+                                ? (long long)a.Hkv * a.B * (a.max_blocks + kSegmentCost) / kMinShareBlocks + 1
                                 : (long long)a.Hkv * a.B * a.max_parts;
     const long long grid = std::max<long long>(1, std::min<long long>((units + C::NW - 1) / C::NW, ctas));
     e = launch_pdl(decode_kernel<C>, dim3((unsigned)grid), dim3(C::NT), smem, st, a);
