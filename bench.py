@@ -186,38 +186,54 @@ TRACES = _Lazy()
 
 # ----------------------------------------------------------------- our arm
 class DeviceStep:
-    """One planned step's metadata as device (or pinned host) tensors."""
+    """One planned step's metadata as device tensors, or (pin=True) packed
+    into one pinned host buffer that to() moves with a single copy."""
+    FIELDS = (("slots", np.int64), ("copies", np.int32), ("tables", np.int32), ("lens", np.int32),
+              ("p_cu", np.int32), ("p_prefix", np.int32), ("p_tables", np.int32))
 
     def __init__(self, plan, torch, device, pin=False):
-        def t(a, dt):
-            x = torch.from_numpy(np.ascontiguousarray(a, dt))
-            if pin:
-                return x.pin_memory()
-            return x.to(device)
-
+        arrs = {"copies": plan.copies, "slots": plan.slots, "tables": plan.decode_tables,
+                "lens": plan.decode_lens, "p_cu": plan.prefill_cu, "p_prefix": plan.prefill_prefix,
+                "p_tables": plan.prefill_tables}
         self.plan = plan
-        self.copies = t(plan.copies, np.int32)
-        self.slots = t(plan.slots, np.int64)
-        self.tables = t(plan.decode_tables, np.int32)
-        self.lens = t(plan.decode_lens, np.int32)
-        self.p_cu = t(plan.prefill_cu, np.int32)
-        self.p_prefix = t(plan.prefill_prefix, np.int32)
-        self.p_tables = t(plan.prefill_tables, np.int32)
+        self.packed = None
+        if pin:
+            # one byte buffer, every field at a 16-byte aligned offset
+            self.layout, off = [], 0
+            for k, dt in self.FIELDS:
+                a = np.ascontiguousarray(arrs[k], dt)
+                self.layout.append((k, dt, off, a.shape))
+                off += (a.nbytes + 15) // 16 * 16
+            host = np.zeros(max(off, 16), np.uint8)
+            for k, dt, o, shape in self.layout:
+                a = np.ascontiguousarray(arrs[k], dt)
+                host[o:o + a.nbytes] = a.view(np.uint8).reshape(-1)
+            self.packed = torch.from_numpy(host).pin_memory()
+        else:
+            for k, dt in self.FIELDS:
+                setattr(self, k, torch.from_numpy(np.ascontiguousarray(arrs[k], dt)).to(device))
         self.T = len(plan.slots)
         self.B = plan.num_decode
         self.nchunks = len(plan.prefill_ids)
         self.pb = 0  # shared prefix blocks attended by cascade decode (0: plain decode)
 
     def to(self, device, non_blocking=True):
+        """Device copy of a packed step: one host-to-device copy, then views."""
+        import torch
         d = object.__new__(DeviceStep)
         d.__dict__.update(self.__dict__)
-        for k in ("copies", "slots", "tables", "lens", "p_cu", "p_prefix", "p_tables"):
-            setattr(d, k, getattr(self, k).to(device, non_blocking=non_blocking))
+        buf = self.packed.to(device, non_blocking=non_blocking)
+        tdt = {np.int32: torch.int32, np.int64: torch.int64}
+        for k, dt, o, shape in self.layout:
+            n = int(np.prod(shape)) * np.dtype(dt).itemsize
+            setattr(d, k, buf[o:o + n].view(tdt[dt]).view(shape))
+        d.packed = None
         return d
 
     def nbytes(self):
-        return sum(getattr(self, k).numel() * getattr(self, k).element_size()
-                   for k in ("copies", "slots", "tables", "lens", "p_cu", "p_prefix", "p_tables"))
+        if self.packed is not None:
+            return self.packed.numel()
+        return sum(getattr(self, k).numel() * getattr(self, k).element_size() for k, _ in self.FIELDS)
 
 
 def run_ours(args, rank, world, device):
