@@ -545,6 +545,7 @@ PA_DEVICE void mma_items(const DecodeArgs &a, const Schedule &sc, Producer<C> &p
             const int s = consumed % C::NSTAGE;
             if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
                 flag_error(a.err, PA_DEVERR_TIMEOUT);
+            __syncwarp();  // the lanes waited separately: converge before the warp-wide MMAs
             const int valid = my_valid[s];
             const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
             // ---- S^T = K q^T

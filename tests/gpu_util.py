@@ -61,3 +61,10 @@ def assert_attn_close(got, ref, what=""):
     mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
     assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}"
     return mx, mean
+
+
+def bf16_round(x):
+    """fp64 values rounded to bf16 (nearest even), back as fp64: the closest
+    a bf16 output can be to the oracle."""
+    t = torch.from_numpy(np.ascontiguousarray(x, np.float64)).to(torch.float32).to(torch.bfloat16)
+    return t.to(torch.float64).numpy()

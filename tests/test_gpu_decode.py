@@ -8,8 +8,8 @@ import pytest
 import torch
 
 import oracle
-from gpu_util import (assert_attn_close, cache_to_device, dev, dev_bf16, dev_u8, host_bits, run_decode,
-                      to_float)
+from gpu_util import (assert_attn_close, bf16_round, cache_to_device, dev, dev_bf16, dev_u8, host_bits,
+                      run_decode, to_float)
 from paged_kv_cache_408_b200 import inputs as I
 from paged_kv_cache_408_b200 import ops
 
@@ -196,4 +196,42 @@ def test_workspace_reuse_across_calls_and_batch_sizes(cuda_device, part):
                    workspace=ws, partition_tokens=part)
         torch.cuda.synchronize()
         assert_attn_close(to_float(out), ref[rows], f"rows {rows.tolist()}")
+    assert ops.get_last_device_error() == 0
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("mag", [0.0, 2.0 ** -80, 2.0 ** -40, 64.0, 1.0e5])
+def test_fp8_gqa8_q_magnitudes(cuda_device, D, mag):
+    """fp8 cache with GQA 8 runs on the tensor cores with q scaled by a power
+    of two into f16 range: all-zero q (uniform softmax: the mean of V), q far
+    below f16's normal range, large q, and q beyond f16's largest value (short
+    sequences, so that the near one-hot softmax has no near ties).
+
+    With large q the softmax is near one-hot and each output is close to one
+    V row, of magnitude up to ~4, where rounding the output to bf16 alone
+    costs up to 2^-9 relative (mean-abs ~1e-3 here, measured against the
+    fp64 oracle with the kernel's arithmetic emulated exactly).  The
+    reference is therefore the oracle rounded to bf16, the closest a bf16
+    output can be; the tolerance is unchanged."""
+    lens = [1, 17, 20] if mag > 1e4 else [1, 15, 16, 33, 200, 513]
+    c = I.make_decode_case(300 + D, lens, 16, 2, D, fp8=True)
+    rng = np.random.default_rng(301)
+    c.q = I.bf16_bits(rng.standard_normal(c.q.shape).astype(np.float32) * np.float32(mag))
+    kc, vc = cache_to_device(c)
+    ref = bf16_round(oracle_decode(c))
+    for part in (0, 16):
+        out = to_float(run_decode(c, kc, vc, partition_tokens=part))
+        assert_attn_close(out, ref, f"|q| x {mag:g}, D{D}, partition {part}")
+    assert ops.get_last_device_error() == 0
+
+
+@pytest.mark.parametrize("Hkv", [1, 3, 4])
+def test_fp8_gqa8_kv_head_counts(cuda_device, Hkv):
+    """fp8 with GQA 8: an even number of kv heads runs warp pairs that share
+    one copy of both heads' block, an odd number one warp per head."""
+    c = I.make_decode_case(320 + Hkv, [1, 16, 17, 100, 700, 1500], 8 * Hkv, Hkv, 128, fp8=True)
+    kc, vc = cache_to_device(c)
+    ref = oracle_decode(c)
+    for part in (0, 32, 512):
+        assert_attn_close(to_float(run_decode(c, kc, vc, partition_tokens=part)), ref, f"Hkv {Hkv} partition {part}")
     assert ops.get_last_device_error() == 0
