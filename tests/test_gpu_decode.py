@@ -227,8 +227,8 @@ def test_fp8_gqa8_q_magnitudes(cuda_device, D, mag):
 
 @pytest.mark.parametrize("Hkv", [1, 3, 4])
 def test_fp8_gqa8_kv_head_counts(cuda_device, Hkv):
-    """fp8 with GQA 8: an even number of kv heads runs warp pairs that share
-    one copy of both heads' block, an odd number one warp per head."""
+    """fp8 with GQA 8 (tensor-core path) with one, an odd and an even number
+    of kv heads, under every partition mode."""
     c = I.make_decode_case(320 + Hkv, [1, 16, 17, 100, 700, 1500], 8 * Hkv, Hkv, 128, fp8=True)
     kc, vc = cache_to_device(c)
     ref = oracle_decode(c)
