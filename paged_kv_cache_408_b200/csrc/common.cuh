@@ -105,6 +105,9 @@ PA_DEVICE void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, ui
 }
 
 // Named barrier `id` (1..15) over `nthreads` threads (a multiple of 32).
+// Fetch the 128-byte line holding p into L2 (no register result, no wait).
+PA_DEVICE void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 PA_DEVICE void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -708,6 +708,14 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     const int gw = blockIdx.x * NW + w, GW = gridDim.x * NW;
     pdl_trigger();  // the merge kernel may be scheduled now; it waits for this grid
     pdl_wait();     // the preceding kernel (e.g. the K/V write) has completed
+    {
+        // bring the block tables and q into L2 while the split is built: the
+        // first bulk copies wait on table entries, the first items on q
+        const size_t tb = (size_t)B * a.max_blocks * sizeof(int32_t), qb = (size_t)B * a.Hq * D * 2;
+        const size_t step = (size_t)gridDim.x * C::NT * 128, o0 = ((size_t)blockIdx.x * C::NT + tid) * 128;
+        for (size_t o = o0; o < tb; o += step) prefetch_l2(reinterpret_cast<const char *>(a.block_tables) + o);
+        for (size_t o = o0; o < qb; o += step) prefetch_l2(static_cast<const char *>(a.q) + o);
+    }
 
     // ---- lengths, then exclusive scans over sequences: the balanced split
     // needs each sequence's offset in the line (Hkv segments of cost units),
