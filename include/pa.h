@@ -201,21 +201,32 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
  * The keys of each sequence split into the shared prefix [0, 16*prefix_blocks)
  * and its own suffix.  The prefix is attended once per kv head for every
  * sequence at the same time (its K/V read once, all sequences' queries as
- * the rows of a tensor-core attention; an fp8 prefix is first widened to
- * bf16 exactly, into the workspace), each suffix by the decode kernel, and
- * the two are combined by the split-K log-sum-exp merge.
+ * the rows of a tensor-core attention, cut into up to 4 key ranges so that
+ * it fills the SMs; an fp8 prefix is first widened to bf16 exactly, into the
+ * workspace), each suffix by the decode kernel, and all pieces are combined
+ * by the split-K log-sum-exp merge.  Four launches (three for bf16), each a
+ * programmatic dependent of the one before, all on `stream`.
  *
- * Arguments as pa_decode (balanced split), plus:
+ * Arguments as pa_decode (balanced split; partition_tokens is not taken),
+ * plus:
  *   prefix_blocks  number of leading block-table entries that every row
  *                  shares: entries 0..prefix_blocks-1 of every row must equal
- *                  those of row 0 (not checked; row 0's are used).  0 runs
+ *                  those of row 0 (not checked; row 0's are used).  Range
+ *                  [0, max_blocks_per_seq] (else PA_ERR_INVALID_ARG); 0 runs
  *                  pa_decode.  Every seq_lens[b] must be >= 16*prefix_blocks
- *                  (checked on the device: PA_DEVERR_BAD_LEN).
- *   workspace      at least pa_decode_cascade_workspace_size() bytes,
- *                  256-byte aligned, no initialisation needed (every call
- *                  writes all it reads).  Calls sharing one workspace must
- *                  not overlap on the GPU.
- * head_dim 64 or 128; bf16 or fp8 E4M3 cache (with k_scale, v_scale).
+ *                  (checked on the device: such a row is flagged
+ *                  PA_DEVERR_BAD_LEN and gets the prefix's attention alone).
+ *   workspace      device memory owned by the caller, at least
+ *                  pa_decode_cascade_workspace_size() bytes, 256-byte
+ *                  aligned (else PA_ERR_WORKSPACE), no initialisation needed
+ *                  (every call writes all it reads).  Calls sharing one
+ *                  workspace must not overlap on the GPU.
+ * head_dim 64 or 128 (else PA_ERR_UNSUPPORTED); num_q_heads / num_kv_heads
+ * in {1,2,4,8}; bf16 or fp8 E4M3 cache (fp8 needs k_scale, v_scale).
+ *
+ * pa_decode_cascade_workspace_size: bytes for num_seqs rows of num_q_heads
+ * heads, tables of max_blocks_per_seq entries and prefix_blocks shared
+ * blocks (an upper bound for any smaller num_seqs); host only.
  */
 int pa_decode_cascade_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t max_blocks_per_seq,
                                      int32_t prefix_blocks, const pa_cache_desc *desc, size_t *bytes);
