@@ -553,15 +553,23 @@ class Scheduler:
         self.step_no += 1
 
     # -- accounting
-    def kv_utilisation(self) -> float:
-        """Stored tokens / capacity of the blocks held by running sequences
-        (shared blocks counted once)."""
+    def kv_accounting(self) -> dict:
+        """Cached tokens of the running sequences (each sequence counted in
+        full) against the distinct blocks they hold: below 1 by the paging
+        waste (under one block per sequence), above 1 where blocks are shared
+        (forks, cached prefixes)."""
         held = set()
         stored = 0
         for s in self.running:
             held.update(s.block_table)
             stored += s.num_cached
-        return stored / (BLOCK_SIZE * len(held)) if held else 1.0
+        return {"sequences": len(self.running), "cached_tokens": stored, "held_blocks": len(held),
+                "tokens_per_block_capacity": stored / (BLOCK_SIZE * len(held)) if held else 1.0}
+
+    def kv_utilisation(self) -> float:
+        """Stored tokens / capacity of the blocks held by running sequences
+        (shared blocks counted once)."""
+        return self.kv_accounting()["tokens_per_block_capacity"]
 
 
 # ------------------------------------------------------------ invariants

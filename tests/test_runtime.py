@@ -297,3 +297,18 @@ def test_forked_trace_shares_its_prompt_blocks_every_step():
     tr = traces.prefix_share_fp8(0, n=24, forks=4, prefix=256)
     for plan in tr.plans(6):
         assert plan.num_decode == 24 and plan.shared_decode_blocks >= 16
+
+
+def test_kv_accounting_shows_paging_waste_and_sharing():
+    from paged_kv_cache_408_b200 import traces
+    tr = traces.batch64_2k(0)
+    tr.plans(5)
+    acc = tr.sched.kv_accounting()
+    assert acc["sequences"] == 64 and 0.9 < acc["tokens_per_block_capacity"] <= 1.0
+    # the waste is below one block per sequence
+    assert acc["held_blocks"] * 16 - acc["cached_tokens"] < 16 * acc["sequences"]
+    tr = traces.prefix_share_fp8(0)
+    tr.plans(2)
+    acc = tr.sched.kv_accounting()
+    # 256 sequences over one 2048-token prefix: each stored token far more often than once
+    assert acc["sequences"] == 256 and acc["tokens_per_block_capacity"] > 5
