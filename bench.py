@@ -790,7 +790,7 @@ def main():
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
             "host_plan_ms_per_step": r["plan_ms"],
-            "kv_accounting": tr.sched.kv_accounting(),
+            "kv_accounting": tr.sched.kv_accounting() if hasattr(tr.sched, "kv_accounting") else None,
             "preemptions": tr.sched.num_preemptions,
         }
         if r["e2e"] is not None:
