@@ -563,8 +563,8 @@ class Scheduler:
         for s in self.running:
             held.update(s.block_table)
             stored += s.num_cached
-        return {"sequences": len(self.running), "cached_tokens": stored, "held_blocks": len(held),
-                "tokens_per_block_capacity": stored / (BLOCK_SIZE * len(held)) if held else 1.0}
+        return {"sequences": len(self.running), "cached_tokens": int(stored), "held_blocks": len(held),
+                "tokens_per_block_capacity": float(stored / (BLOCK_SIZE * len(held))) if held else 1.0}
 
     def kv_utilisation(self) -> float:
         """Stored tokens / capacity of the blocks held by running sequences

@@ -312,3 +312,5 @@ def test_kv_accounting_shows_paging_waste_and_sharing():
     acc = tr.sched.kv_accounting()
     # 256 sequences over one 2048-token prefix: each stored token far more often than once
     assert acc["sequences"] == 256 and acc["tokens_per_block_capacity"] > 5
+    import json
+    json.dumps(acc)  # bench.py prints it in its JSON line
