@@ -325,30 +325,33 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
 
-    # ---- warm-up
-    for ds in dsteps[:args.warmup]:
-        launch(ds, q, out, new_k, new_v, pq, pout)
-        decode(ds, q, out)
-        prefill(ds, pq, pout)
-    torch.cuda.synchronize()
-    if ops.get_last_device_error() != 0:
-        raise RuntimeError("device status word set during warm-up")
-
-    # ---- timed: inputs resident in HBM, L2 flushed between steps (outside the events)
-    timed = dsteps[args.warmup:]
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
-    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
-    launches = 0
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        # ---- warm-up, with the clock sampler already running: its start-up pause
+        # must not leave the GPU idle (clocks falling back) right before the
+        # timed steps; the warm-up steps flush L2 like the timed ones
+        for ds in dsteps[:args.warmup]:
+            flush()
+            launch(ds, q, out, new_k, new_v, pq, pout)
+            decode(ds, q, out)
+            prefill(ds, pq, pout)
+        torch.cuda.synchronize()
+        if ops.get_last_device_error() != 0:
+            raise RuntimeError("device status word set during warm-up")
+
+        # ---- timed: inputs resident in HBM, L2 flushed between steps (outside the events)
+        timed = dsteps[args.warmup:]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
+        dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
+        launches = 0
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
         # hold the stream while the host enqueues every timed step, so the
         # events see device time only (no host launch gaps).  Only the step
         # is bracketed: an event between two kernels would cut the
         # programmatic launch chain (write -> decode -> merge -> prefill).
-        torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
+        torch.cuda._sleep(hold_cycles(len(timed)))
         for ds, (e0, e1) in zip(timed, ev):
             flush()
             e0.record(st)
@@ -359,7 +362,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize()
         # the decode call alone (its kernel and the merge), same steps and
         # cache, for the roofline of the dominant kernel
-        torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
+        torch.cuda._sleep(hold_cycles(len(timed)))
         for ds, (e0, e1) in zip(timed, dev_ev):
             flush()
             e0.record(st)
@@ -368,7 +371,7 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize()
         sfx_ev = []
         if any(ds.pb for ds in timed):
-            torch.cuda._sleep(int(2e7 + 1e6 * len(timed)))
+            torch.cuda._sleep(hold_cycles(len(timed)))
             for ds in timed:
                 if ds.B and ds.pb:
                     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -518,7 +521,7 @@ def run_mixed(args, rank, world, device):
     def timed(fn, n):
         """n calls of fn, each bracketed by events, L2 flushed in between."""
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        torch.cuda._sleep(int(2e7 + 1e6 * n))
+        torch.cuda._sleep(hold_cycles(n))
         for e0, e1 in ev:
             flush()
             e0.record(st)
@@ -665,6 +668,14 @@ def aggregate(tot_s, kv_bytes_done, seq_steps, world, device):
     dist.all_reduce(w, op=dist.ReduceOp.SUM)
     return float(t.item()), float(w[0].item()), float(w[1].item())
 
+
+
+def hold_cycles(n_steps):
+    """GPU clock cycles of the sleep that holds the stream while the host
+    enqueues n timed steps (outside the timed events): about 10 ms plus
+    0.5 ms a step at 1.965 GHz, well above the enqueue time (tens of us a
+    step)."""
+    return int(2e7 + 1e6 * n_steps)
 
 
 def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload, cuda_core_math=True):
