@@ -530,14 +530,17 @@ def run_mixed(args, rank, world, device):
         torch.cuda.synchronize()
         return [e0.elapsed_time(e1) for e0, e1 in ev]
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
+    # the clock sampler starts before the warm-up: its start-up pause must not
+    # leave the GPU idle right before the timed steps
     with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.warmup):
+            flush()
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
         step_ms = timed(step, args.steps)  # the whole step: one programmatic launch chain
         dec_ms = timed(decode, args.steps)  # then each kernel alone, for its roofline
         pre_ms = timed(prefill, args.steps)
