@@ -446,7 +446,7 @@ def run_ours(args, rank, world, device):
 
     return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb, algf=algf,
                 launches=launches, clocks=clk.summary(), e2e=e2e, plan_ms=t_plan * 1e3, tr=tr, plans=plans,
-                cascade=cascade,
+                cascade=cascade, copies=sum(len(ds.plan.copies) for ds in timed),
                 k_cache=k_cache, v_cache=v_cache, Hq=Hq, Hkv=Hkv, D=D, eb=eb, fp8=fp8, scale=scale,
                 k_scale=k_scale, v_scale=v_scale, q=q, pool=pool)
 
@@ -805,6 +805,7 @@ def main():
             "clocks": r["clocks"],
             "host_plan_ms_per_step": r["plan_ms"],
             "kv_accounting": tr.sched.kv_accounting() if hasattr(tr.sched, "kv_accounting") else None,
+            "blocks_copied_per_step": r.get("copies", 0) / args.steps,
             "preemptions": tr.sched.num_preemptions,
         }
         if r["e2e"] is not None:
