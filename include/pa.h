@@ -83,7 +83,7 @@ typedef enum pa_dtype {
 /* Bits of the device status word (pa_get_last_device_error). */
 #define PA_DEVERR_BAD_BLOCK 0x1u  /* a block-table entry outside [0, num_blocks) was needed */
 #define PA_DEVERR_BAD_SLOT 0x2u   /* a slot mapped past the last block */
-#define PA_DEVERR_BAD_LEN 0x4u    /* seq_len < 0 or > 16 * max_blocks_per_seq */
+#define PA_DEVERR_BAD_LEN 0x4u    /* seq_len < 0 or > 16 * max_blocks_per_seq (cascade: < 16 * prefix_blocks) */
 #define PA_DEVERR_BAD_PAIR 0x8u   /* a copy pair outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait for an async copy or MMA gave up (results invalid) */
 
@@ -309,7 +309,8 @@ int pa_get_last_device_error(uint32_t *flags, pa_stream_t stream);
 /* Human-readable name of a pa_status value (static string). */
 const char *pa_status_string(int status);
 
-/* Library version as an integer (major*10000 + minor*100 + patch). */
+/* Library version as an integer (major*10000 + minor*100 + patch): 200 =
+ * 0.2.0, which adds pa_decode_cascade and pa_decode_noalloc to 0.1.0. */
 int pa_version(void);
 
 #ifdef __cplusplus

@@ -62,7 +62,7 @@ unsigned *pa::status_word() { return status_word_ptr(); }
 
 extern "C" {
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 200; }
 
 const char *pa_status_string(int status) {
     switch (status) {
