@@ -150,6 +150,12 @@ def decode_alg_flops(lens, Hq, D):
     return 4 * D * Hq * int(np.asarray(lens, np.int64).sum())
 
 
+def roof_time(nbytes, bytes_per_s, flops, flops_per_s):
+    """Shortest time for work that moves nbytes and does flops: the slower of
+    the memory roof and the arithmetic roof."""
+    return max(nbytes / bytes_per_s, flops / flops_per_s)
+
+
 def decode_math_on_cuda_cores(Hq, Hkv, fp8):
     """The decode kernel does q.k and p.v on the CUDA cores except for an fp8
     cache with GQA 8, where it uses the tensor cores (mma.sync, f16)."""
@@ -695,8 +701,8 @@ def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload, cuda_core_m
               "peak_kind": tkind, "kernel": "prefill_kernel (shared-prefix mode) + fp8 widening",
               "ms_per_launch": t_pre * 1e3, "alg_flops_per_launch": c["prefix_flops"],
               "timing": "cascade call minus the suffix stage timed alone", "traffic": None}
-    alu_s = c["suffix_flops"] / (apeak * 1e12) if cuda_core_math else c["suffix_flops"] / (tpeak * 1e12)
-    if cuda_core_math and alu_s > c["suffix_bytes"] / (hbm_peak * 1e9):
+    sfx_flops_per_s = (apeak if cuda_core_math else tpeak) * 1e12
+    if cuda_core_math and c["suffix_flops"] / sfx_flops_per_s > c["suffix_bytes"] / (hbm_peak * 1e9):
         tfl = c["suffix_flops"] / t_sfx / 1e12
         suffix = {"bound": "alu", "achieved": tfl, "peak": apeak, "unit": "TFLOP/s", "frac": tfl / apeak,
                   "peak_kind": f"derived: 148 SMs x 128 fp32 lanes x 2 FLOP x {sm_mhz:.0f} MHz"}
@@ -709,7 +715,7 @@ def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload, cuda_core_m
                    "timing": "decode call over the suffix tables, CUDA events",
                    "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", workload + ":suffix")})
     roof_s = (c["prefix_flops"] / (tpeak * 1e12) +
-              max(alu_s, c["suffix_bytes"] / (hbm_peak * 1e9)))
+              roof_time(c["suffix_bytes"], hbm_peak * 1e9, c["suffix_flops"], sfx_flops_per_s))
     out = dict(suffix if t_sfx >= t_pre else prefix)
     out["stages"] = {"prefix": prefix, "suffix": suffix,
                      "call": {"ms_per_launch": t_call * 1e3, "roof_ms": roof_s * 1e3, "frac": roof_s / t_call,
@@ -777,7 +783,7 @@ def main():
         sm_mhz = (r["clocks"] or {}).get("sm_mhz") or 1965.0
         apeak = alu_peak(sm_mhz)
         cuda_core_math = decode_math_on_cuda_cores(r.get("Hq", 32), r.get("Hkv", 8), r["fp8"])
-        alu_bound = cuda_core_math and flops / (apeak * 1e12) > alg / (peak * 1e9)
+        alu_bound = cuda_core_math and roof_time(alg, peak * 1e9, flops, apeak * 1e12) > alg / (peak * 1e9)
         if alu_bound:
             tfl = flops / (dec_ms / 1e3) / 1e12
             roof = {"bound": "alu", "achieved": tfl, "peak": apeak, "unit": "TFLOP/s", "frac": tfl / apeak,

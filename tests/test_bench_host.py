@@ -67,3 +67,25 @@ def test_packed_step_metadata_round_trips(monkeypatch):
         for k, _ in bench.DeviceStep.FIELDS:
             a, b = getattr(plain, k), getattr(moved, k)
             assert a.dtype == b.dtype and a.shape == b.shape and torch.equal(a, b), k
+
+
+def test_roof_time_reproduces_the_pages_batching_model():
+    """The two-roof bound bench.py uses, checked against the batching table of
+    the third page (pass time and tokens/s for B sequences sharing one read of
+    the weights; tests/golden/batching_model.json cites it).  Summing the two
+    roofs instead of taking the slower, or swapping bytes and FLOPs, breaks
+    the small-batch rows or the plateau."""
+    import json
+    import os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "batching_model.json")))
+    m = g["model"]
+    for row in g["rows"]:
+        B = row["batch"]
+        t = bench.roof_time(m["weight_bytes"], m["hbm_bytes_per_s"], B * m["flops_per_token"],
+                            m["usable_fraction"] * m["peak_flops_per_s"])
+        assert abs(t * 1e3 - row["pass_ms"]) <= 0.06, (B, t)   # printed to 0.1 ms
+        assert B / t == pytest.approx(row["tokens_per_s"], rel=0.01)
+    # the crossover: memory-bound up to 26 sequences, compute-bound beyond
+    w = m["weight_bytes"] / m["hbm_bytes_per_s"]
+    per = m["flops_per_token"] / (m["usable_fraction"] * m["peak_flops_per_s"])
+    assert int(w // per) == 25 and w / per < 26
