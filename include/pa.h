@@ -160,12 +160,12 @@ int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head
  *   seq_lens      int32 [num_seqs]; 0 gives an all-zero output row.
  *   scale         softmax scale (typically 1/sqrt(head_dim)).
  *   k_scale, v_scale  fp32 [num_kv_heads] for an fp8 cache, else ignored.
- *   partition_tokens  how a sequence's tokens are split across CTAs
+ *   partition_tokens  how a sequence's tokens are split across warps
  *                 (split-K; the pieces are combined by a log-sum-exp merge
- *                 inside the same kernel):
+ *                 kernel that the same call enqueues):
  *                 0  -- balanced: the (sequence, kv head, block) work of the
  *                       whole batch is cut into equal contiguous shares, one
- *                       per resident CTA, so every SM streams the same
+ *                       per resident warp, so every SM streams the same
  *                       number of bytes whatever the length mix (fastest;
  *                       split points depend on the batch, so the last bits
  *                       of a result can differ between batch compositions);
@@ -181,7 +181,10 @@ int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head
  *                 keeps nothing between calls.  Calls that share one
  *                 workspace must not overlap on the GPU.
  * num_seqs must be in [0, 2048] (0 enqueues nothing); num_kv_heads <= 128;
- * num_q_heads / num_kv_heads in {1,2,4,8}.
+ * num_q_heads / num_kv_heads in {1,2,4,8}.  With an fp8 cache and 8 q heads
+ * per kv head the products run on the tensor cores (f16 operands: E4M3
+ * exactly, q scaled by a power of two; fp32 accumulation), otherwise in fp32
+ * on the CUDA cores.
  */
 int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache, const int32_t *block_tables,
               const int32_t *seq_lens, int32_t num_seqs, int32_t max_blocks_per_seq, int32_t num_q_heads,
