@@ -65,6 +65,10 @@ extern "C" {
 
 #define PA_BLOCK_SIZE 16
 
+/* Largest max_blocks_per_seq any call accepts (2^24 blocks = 2^28 tokens per
+ * sequence); wider tables return PA_ERR_INVALID_ARG. */
+#define PA_MAX_BLOCKS_PER_SEQ (1 << 24)
+
 typedef enum pa_status {
     PA_OK = 0,
     PA_ERR_INVALID_ARG = -1, /* null pointer, bad size, Hq % Hkv != 0, block_size != 16 */

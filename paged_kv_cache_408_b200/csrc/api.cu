@@ -60,6 +60,16 @@ int resolve_partition(int32_t partition_tokens, int *out) {
 
 unsigned *pa::status_word() { return status_word_ptr(); }
 
+int pa::sm_count() {
+    static std::mutex mu;
+    static int n[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!n[dev] && cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n[dev] = 0;
+    return n[dev] > 0 ? n[dev] : 1;
+}
+
 extern "C" {
 
 int pa_version(void) { return 200; }
@@ -108,7 +118,9 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, i
 
 int pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim, int32_t max_blocks_per_seq,
                              int32_t partition_tokens, size_t *bytes) {
-    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
+    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 ||
+        max_blocks_per_seq > pa::kMaxBlocksPerSeq)
+        return PA_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
     int P = 0;
     int rc = resolve_partition(partition_tokens, &P);
@@ -124,7 +136,8 @@ int pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache
               void *workspace, size_t workspace_bytes, const pa_cache_desc *desc, pa_stream_t stream) {
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
-    if (num_seqs < 0 || num_seqs > kMaxSeqs || max_blocks_per_seq <= 0 || num_q_heads <= 0)
+    if (num_seqs < 0 || num_seqs > kMaxSeqs || max_blocks_per_seq <= 0 ||
+        max_blocks_per_seq > pa::kMaxBlocksPerSeq || num_q_heads <= 0)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (desc->num_kv_heads > pa::kMaxDecodeKvHeads) return PA_ERR_UNSUPPORTED;
@@ -155,8 +168,8 @@ int pa_decode_cascade_workspace_size(int32_t num_seqs, int32_t num_q_heads, int3
                                      int32_t prefix_blocks, const pa_cache_desc *desc, size_t *bytes) {
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
-    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 || prefix_blocks < 0 ||
-        prefix_blocks > max_blocks_per_seq)
+    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || max_blocks_per_seq <= 0 ||
+        max_blocks_per_seq > pa::kMaxBlocksPerSeq || prefix_blocks < 0 || prefix_blocks > max_blocks_per_seq)
         return PA_ERR_INVALID_ARG;
     *bytes = pa::cascade_ws_bytes(num_seqs, num_q_heads, desc->num_kv_heads, desc->head_dim, max_blocks_per_seq,
                                   prefix_blocks, desc->dtype == PA_DTYPE_FP8_E4M3);
@@ -170,7 +183,8 @@ int pa_decode_cascade(void *out, const void *q, const void *k_cache, const void 
                       const pa_cache_desc *desc, pa_stream_t stream) {
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
-    if (num_seqs < 0 || num_seqs > kMaxSeqs || max_blocks_per_seq <= 0 || num_q_heads <= 0)
+    if (num_seqs < 0 || num_seqs > kMaxSeqs || max_blocks_per_seq <= 0 ||
+        max_blocks_per_seq > pa::kMaxBlocksPerSeq || num_q_heads <= 0)
         return PA_ERR_INVALID_ARG;
     if (prefix_blocks < 0 || prefix_blocks > max_blocks_per_seq) return PA_ERR_INVALID_ARG;
     if (prefix_blocks == 0)  // nothing shared: plain decode
@@ -203,7 +217,8 @@ int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const i
     (void)v_scale;
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
-    if (num_chunks < 0 || max_blocks_per_seq <= 0 || num_q_heads <= 0 || max_q_len < 0 || total_q_tokens < 0)
+    if (num_chunks < 0 || max_blocks_per_seq <= 0 || max_blocks_per_seq > pa::kMaxBlocksPerSeq ||
+        num_q_heads <= 0 || max_q_len < 0 || total_q_tokens < 0)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int G = num_q_heads / desc->num_kv_heads;

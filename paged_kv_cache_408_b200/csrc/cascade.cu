@@ -25,7 +25,6 @@ namespace pa {
 namespace {
 
 size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
-constexpr int kNumSMs = 148;
 
 // Widen the prefix blocks of both caches (block_tables row 0) to bf16 into
 // [prefix_blocks][Hkv][16][D] scratch and write the identity table.  One
@@ -102,7 +101,7 @@ cudaError_t launch_decode_cascade(const DecodeArgs &d, void *workspace, cudaStre
     {
         const int ctas = a.Hkv * ((a.B * (a.Hq / a.Hkv) + 255) / 256);
         const int tiles = (p.shared_len + 127) / 128;
-        p.key_splits = std::max(1, std::min({kNumSMs / std::max(ctas, 1), kMaxPrefixSplits, tiles}));
+        p.key_splits = std::max(1, std::min({sm_count() / std::max(ctas, 1), kMaxPrefixSplits, tiles}));
     }
     a.prefix_pieces = p.key_splits;
     cudaError_t e = cudaSuccess;
@@ -114,7 +113,7 @@ cudaError_t launch_decode_cascade(const DecodeArgs &d, void *workspace, cudaStre
         uint4 *vout = reinterpret_cast<uint4 *>(reinterpret_cast<char *>(kout) +
                                                round256((size_t)a.prefix_blocks * block_elems * 2));
         const int64_t n8 = (int64_t)a.prefix_blocks * block_elems / 8;
-        const unsigned grid = (unsigned)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
+        const unsigned grid = (unsigned)std::min<int64_t>((n8 + 255) / 256, (int64_t)sm_count() * 8);
         e = launch_pdl(widen_prefix_kernel, dim3(grid), dim3(256), 0, st, static_cast<const uint8_t *>(a.k_cache),
                        static_cast<const uint8_t *>(a.v_cache), a.block_tables, a.prefix_blocks, a.num_blocks,
                        block_elems, kout, vout, ident, a.err);

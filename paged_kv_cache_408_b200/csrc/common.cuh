@@ -53,14 +53,25 @@ PA_DEVICE uint64_t global_ns() {
     return t;
 }
 
-// Wait for phase `parity` of `bar` to complete.  The wait is bounded: after
-// about `limit_ns` nanoseconds it gives up and returns false, so a lost
-// transaction can never hang the GPU; the caller records PA_DEVERR_TIMEOUT.
-PA_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
+// Bounded waits.  Every wait of a launch shares ONE deadline, taken once per
+// thread right after the launch's dependency wait (wait_deadline()), so a
+// lost transaction ends the whole launch about kWaitBudgetNs after it
+// started, however many waits remain.  Callers stop issuing waits after the
+// first failure (they evaluate `ok && mbar_wait(...)`), record
+// PA_DEVERR_TIMEOUT, then drain what they have in flight with
+// drain_deadline(): a short fresh budget for the copies and MMAs already
+// issued, so that no asynchronous write lands after the CTA has exited.
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;   // 2 s per launch
+constexpr uint64_t kDrainBudgetNs = 20000000ull;    // 20 ms for the drain after a failure
+
+PA_DEVICE uint64_t wait_deadline() { return global_ns() + kWaitBudgetNs; }
+PA_DEVICE uint64_t drain_deadline() { return global_ns() + kDrainBudgetNs; }
+
+// Wait for phase `parity` of `bar` to complete, until `deadline` (ns of
+// %globaltimer); false if the deadline passed first.
+PA_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t deadline) {
     while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > limit_ns) return false;
+        if (global_ns() > deadline) return false;
     return true;
 }
 

@@ -382,6 +382,20 @@ struct Producer {
     }
 };
 
+// After a wait of this warp's ring ran past the launch deadline: record the
+// timeout, stop streaming, and wait (with a short fresh budget) for the
+// copies this warp has issued but not consumed, so that none lands in
+// shared memory after the warp has exited.  Each of those stages has exactly
+// one copy in flight (a stage is refilled only after it was consumed).
+template <class C>
+PA_DEVICE void give_up(const DecodeArgs &a, uint64_t *bars, uint32_t consumed, uint32_t issued, int lane) {
+    if (lane == 0) flag_error(a.err, PA_DEVERR_TIMEOUT);
+    const uint64_t dd = drain_deadline();
+    for (uint32_t c = consumed; c < issued; ++c)
+        if (!mbar_wait(&bars[c % C::NSTAGE], (c / C::NSTAGE) & 1, dd)) break;
+    __syncwarp();
+}
+
 // Load this lane's chunks of one token row from shared memory and widen to fp32 pairs.
 template <class C>
 PA_DEVICE void load_row(const uint8_t *row, const int (&choff)[C::NCH], float2 (&f)[C::P2]) {
@@ -498,7 +512,7 @@ struct QPrefetchMma {
 template <class C>
 PA_DEVICE void mma_items(const DecodeArgs &a, const Schedule &sc, Producer<C> &prod, ItemIter &items,
                          uint8_t *my_stages, uint64_t *my_bars, int *my_valid, int lane, const uint8_t *kc,
-                         const uint8_t *vc) {
+                         const uint8_t *vc, uint64_t deadline) {
     constexpr int D = C::D, G = C::G, NK = D / 16, NM = D / 16, KW = D / 16, VB = D / 8;
     static_assert(C::FP8 && G == 8, "tensor-core decode: fp8 cache, GQA 8");
     const int r = lane >> 2, c = lane & 3, Hkv = sc.Hkv;
@@ -543,9 +557,11 @@ PA_DEVICE void mma_items(const DecodeArgs &a, const Schedule &sc, Producer<C> &p
 
         for (int j = 0; j < it.nblk; ++j) {
             const int s = consumed % C::NSTAGE;
-            if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
-                flag_error(a.err, PA_DEVERR_TIMEOUT);
-            __syncwarp();  // the lanes waited separately: converge before the warp-wide MMAs
+            // the lanes waited separately: agree (and converge) before the warp-wide MMAs
+            if (!__all_sync(kFull, mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1, deadline))) {
+                give_up<C>(a, my_bars, consumed, prod.issued, lane);
+                return;
+            }
             const int valid = my_valid[s];
             const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
             // ---- S^T = K q^T
@@ -708,6 +724,7 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     const int gw = blockIdx.x * NW + w, GW = gridDim.x * NW;
     pdl_trigger();  // the merge kernel may be scheduled now; it waits for this grid
     pdl_wait();     // the preceding kernel (e.g. the K/V write) has completed
+    const uint64_t deadline = wait_deadline();  // shared by every wait of this launch
     {
         // bring the block tables and q into L2 while the split is built: the
         // first bulk copies wait on table entries, the first items on q
@@ -829,7 +846,7 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
     ItemIter items;
     items.start(sc, gw, GW);
     if constexpr (C::MMA) {
-        mma_items<C>(a, sc, prod, items, my_stages, my_bars, my_valid, lane, kc, vc);
+        mma_items<C>(a, sc, prod, items, my_stages, my_bars, my_valid, lane, kc, vc, deadline);
     } else {
         Item it, nx;
         bool have = items.next(sc, it);
@@ -862,8 +879,10 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
 
             for (int j = 0; j < it.nblk; ++j) {
                 const int s = consumed % C::NSTAGE;
-                if (!mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1) && lane == 0)
-                    flag_error(a.err, PA_DEVERR_TIMEOUT);
+                if (!__all_sync(kFull, mbar_wait(&my_bars[s], (consumed / C::NSTAGE) & 1, deadline))) {
+                    give_up<C>(a, my_bars, consumed, prod.issued, lane);
+                    return;
+                }
                 const int valid = my_valid[s];
                 const uint8_t *Kb = my_stages + (size_t)s * 2 * C::BLKB, *Vb = Kb + C::BLKB;
 
@@ -1016,10 +1035,14 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
 // as a programmatic dependent of the decode kernel: its CTAs may become
 // resident while the decode grid drains, and griddepcontrol.wait returns
 // once that grid has completed with its memory visible.  Lane l owns head
-// dims [l*E, l*E + E).  The length, the piece count and the first kFirst
-// pieces are loaded together (addresses do not depend on the count; slots
-// past it are in bounds and ignored), so up to kFirst pieces cost one L2
-// round trip.
+// dims [l*E, l*E + E).  The length, the piece count and the first
+// merge_spec pieces are loaded together (their addresses do not depend on
+// the count), so a row of up to merge_spec pieces costs one L2 round trip;
+// the launcher picks merge_spec so that those slots are written for every
+// row that needs a merge (a cascade's prefix pieces and its first suffix
+// piece; 2 in plain decode), so the look-ahead never reads a stale slot
+// (after an L2 flush, from DRAM).  The rest of a row's pieces are loaded
+// once its count is known.
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
     constexpr int E = D / 32, kFirst = 8;
@@ -1046,10 +1069,11 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
     };
     const int len = __ldcg(a.seq_lens + b);
     const int np = __ldcg(a.ws_np + (size_t)b * a.Hkv + kvh);
+    const int spec = a.merge_spec;  // <= min(kFirst, max_parts)
     float lp[kFirst], v[kFirst][E];
 #pragma unroll
     for (int u = 0; u < kFirst; ++u)
-        if (u < a.max_parts) {
+        if (u < spec) {
             lp[u] = __ldcg(lse + u);
             load_o(u, v[u]);
         }
@@ -1065,14 +1089,12 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
     for (int p0 = 0; p0 < np; p0 += kFirst) {
-        if (p0 > 0) {
 #pragma unroll
-            for (int u = 0; u < kFirst; ++u)
-                if (p0 + u < np) {
-                    lp[u] = __ldcg(lse + p0 + u);
-                    load_o(p0 + u, v[u]);
-                }
-        }
+        for (int u = 0; u < kFirst; ++u)
+            if (p0 + u < np && (p0 > 0 || u >= spec)) {
+                lp[u] = __ldcg(lse + p0 + u);
+                load_o(p0 + u, v[u]);
+            }
         float mc = M;
 #pragma unroll
         for (int u = 0; u < kFirst; ++u)
@@ -1148,7 +1170,12 @@ cudaError_t run(const DecodeArgs &a, cudaStream_t st) {
     e = launch_pdl(decode_kernel<C>, dim3((unsigned)grid), dim3(C::NT), smem, st, a);
     if (e != cudaSuccess || !a.ws_np) return e;  // no workspace: every (sequence, kv head) is one piece
     const long long rows = (long long)a.B * a.Hq;
-    return launch_pdl(merge_kernel<C::D>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st, a);
+    DecodeArgs m = a;
+    // pieces every merged row is sure to have: a cascade row has its prefix
+    // pieces and (unless its suffix is empty) one suffix piece; a plain row
+    // that needs a merge has at least two
+    m.merge_spec = std::min({8, a.max_parts, a.prefix_blocks ? a.prefix_pieces + 1 : 2});
+    return launch_pdl(merge_kernel<C::D>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st, m);
 }
 
 template <int D, bool FP8>

@@ -48,7 +48,8 @@ extern "C" int pa_decode_noalloc(void *out, const void *q, const void *k_cache, 
         return PA_ERR_INVALID_ARG;
     if (desc->dtype != PA_DTYPE_BF16 && desc->dtype != PA_DTYPE_FP8_E4M3) return PA_ERR_INVALID_ARG;
     if (desc->head_dim != 64 && desc->head_dim != 128) return PA_ERR_UNSUPPORTED;
-    if (num_seqs < 0 || num_seqs > pa::kMaxDecodeSeqs || max_blocks_per_seq <= 0 || num_q_heads <= 0)
+    if (num_seqs < 0 || num_seqs > pa::kMaxDecodeSeqs || max_blocks_per_seq <= 0 ||
+        max_blocks_per_seq > pa::kMaxBlocksPerSeq || num_q_heads <= 0)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     if (desc->num_kv_heads > pa::kMaxDecodeKvHeads) return PA_ERR_UNSUPPORTED;

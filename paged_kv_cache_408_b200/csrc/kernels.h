@@ -49,6 +49,8 @@ struct DecodeArgs {
     int prefix_blocks;     // cascade: the first prefix_blocks of every row are attended elsewhere (pieces
                            // 0..prefix_pieces-1); this launch attends the rest as the pieces after them (0: off)
     int prefix_pieces;
+    int merge_spec;        // pieces the merge kernel loads per row before it has read the row's piece count
+                           // (set by the decode launcher)
 };
 
 struct PrefillArgs {
@@ -84,6 +86,10 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st);
 // Device address of the status word on the current device (nullptr if unknown).
 unsigned *status_word();
 
+// Streaming multiprocessors of the current device (queried once per device
+// and cached; 148 on a B200).  Grids are sized in multiples of it.
+int sm_count();
+
 // Workspace layout shared by pa_decode_workspace_size, pa_decode and
 // pa_decode_noalloc: [piece counts | partial outputs | partial log2-sum-exp],
 // each region 256-byte aligned.  Every call writes what it reads (the decode
@@ -92,10 +98,14 @@ unsigned *status_word();
 constexpr int kMaxDecodeSeqs = 2048;
 constexpr int kMinShareBlocks = 16;  // balanced split: smallest per-warp share, in cost units
 constexpr int kMaxDecodeKvHeads = 128;
-// Pieces one (sequence, kv head) of max_blocks blocks can be cut into.
+// Widest block table any entry point accepts (PA_MAX_BLOCKS_PER_SEQ): token
+// positions (16 * max_blocks) and piece counts stay far inside int32.
+constexpr int kMaxBlocksPerSeq = PA_MAX_BLOCKS_PER_SEQ;
+// Pieces one (sequence, kv head) of max_blocks blocks can be cut into
+// (max_blocks in [1, kMaxBlocksPerSeq], checked by every entry point).
 inline int decode_max_parts(int max_blocks, int partition_tokens) {
-    return partition_tokens == 0 ? max_blocks / kMinShareBlocks + 2
-                                 : (max_blocks * 16 + partition_tokens - 1) / partition_tokens;
+    const int64_t mb = max_blocks;
+    return (int)(partition_tokens == 0 ? mb / kMinShareBlocks + 2 : (mb * 16 + partition_tokens - 1) / partition_tokens);
 }
 size_t decode_ws_bytes(int B, int Hq, int D, int max_parts);
 // Points a.ws_np / a.ws_o / a.ws_lse into a workspace of decode_ws_bytes().

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int i0 = blockIdx.x * (NQ * C::QPOS);
     pdl_trigger();
     pdl_wait();
+    const uint64_t deadline = wait_deadline();  // shared by every wait of this launch
     // causal chunk: rows are positions pfx + i, keys [0, pfx + i]; shared
     // prefix: rows are sequences, keys [0, shared_len) for every row
     const bool shared = a.shared_len > 0;
@@ -180,7 +181,19 @@ __global__ void __launch_bounds__(C::NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // ok turns false at the first wait that runs past the deadline; after
+    // that no role issues another wait of the protocol: the loader and the
+    // MMA warp stop issuing, the softmax warps only keep their named
+    // barriers and arrivals in step (so no thread waits on a partner that has
+    // left), and the asynchronous work already issued is drained below.
+    // ok is kept warp-uniform, since tcgen05.ld/st and the MMA issue are
+    // warp-collective.
     bool ok = true;
+    auto wait = [&](uint64_t *bar, uint32_t parity) {
+        ok = ok && mbar_wait(bar, parity, deadline);
+        ok = __all_sync(0xffffffffu, ok);
+        return ok;
+    };
 
     if (w == C::W_LOAD) {
         // ---- producer: K tile j, then V tile j, into ring slot j % NS.  The
@@ -189,7 +202,8 @@ __global__ void __launch_bounds__(C::NT, 1)
         // copies are issued without a global round trip.
         constexpr int BPT = KT / 16;  // blocks per tile
         int win0 = jt0 * BPT, went = bt[min(win0 + lane, nalloc - 1)];
-        for (int j = 0; j < ntiles; ++j) {
+        int kissued = 0, vissued = 0;  // tiles whose K / V copies were issued
+        for (int j = 0; j < ntiles && ok; ++j) {
             const int s = j % NS, jb = (jt0 + j) * BPT;  // first block of the tile
             const uint32_t use = j / NS;  // how many times slot s was filled before
             if (jb + BPT > win0 + 32) {
@@ -206,7 +220,8 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
             for (int kv = 0; kv < 2; ++kv) {
                 uint64_t *full = kv ? &vfull[s] : &kfull[s];
-                if (use > 0) ok = mbar_wait(kv ? &vempty[s] : &kempty[s], (use - 1) & 1) && ok;
+                if (use > 0 && !wait(kv ? &vempty[s] : &kempty[s], (use - 1) & 1)) break;
+                (kv ? vissued : kissued) = j + 1;
                 if (lane == 0) mbar_arrive_expect_tx(full, C::TX_BYTES);
                 __syncwarp();
                 if (lane < BPT) {
@@ -217,6 +232,17 @@ __global__ void __launch_bounds__(C::NT, 1)
                 }
                 __syncwarp();
             }
+        }
+        if (!ok) {
+            // each slot has at most one copy in flight (a slot is refilled only
+            // after its previous fill was consumed): wait for the last fill of
+            // every slot, with a short fresh budget
+            const uint64_t dd = drain_deadline();
+            for (int sl = 0; sl < NS; ++sl) {
+                if (kissued > sl) mbar_wait(&kfull[sl], ((kissued - 1 - sl) / NS) & 1, dd);
+                if (vissued > sl) mbar_wait(&vfull[sl], ((vissued - 1 - sl) / NS) & 1, dd);
+            }
+            __syncwarp();
         }
     } else if (w == C::W_MMA) {
         // ---- MMA issue, software-pipelined per query tile: O_t += P_t(j) V_j
@@ -238,17 +264,16 @@ __global__ void __launch_bounds__(C::NT, 1)
             }
             __syncwarp();
         };
-        if (ntiles > 0) {
-            ok = mbar_wait(&kfull[0], 0) && ok;
+        if (ntiles > 0 && wait(&kfull[0], 0)) {
 #pragma unroll
             for (int t = 0; t < NQ; ++t)
                 if (ntl[t] > 0) issue_s(t, 0);
             if (lane == 0) tc_commit(&kempty[0]);
             __syncwarp();
         }
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; j < ntiles && ok; ++j) {
             const int s = j % NS, jn = j + 1, sn = jn % NS;
-            ok = mbar_wait(&vfull[s], (j / NS) & 1) && ok;
+            if (!wait(&vfull[s], (j / NS) & 1)) break;
             const int kv0 = (jt0 + j) * KT;
             if (kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
                 uint8_t *vt = sV + s * C::KTILE;
@@ -265,7 +290,7 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
             for (int t = 0; t < NQ; ++t) {
                 if (j < ntl[t]) {
-                    ok = mbar_wait(&pfull[t], j & 1) && ok;  // P_t(j) is in TMEM
+                    if (!wait(&pfull[t], j & 1)) break;  // P_t(j) is in TMEM
                     if (lane == 0) {
                         tc_fence_after();
                         const uint32_t v0 = smem_addr(sV + s * C::KTILE);
@@ -281,25 +306,28 @@ __global__ void __launch_bounds__(C::NT, 1)
                 }
                 if (jn < ntl[t]) {
                     if (!kready) {
-                        ok = mbar_wait(&kfull[sn], (jn / NS) & 1) && ok;
+                        if (!wait(&kfull[sn], (jn / NS) & 1)) break;
                         kready = true;
                     }
-                    ok = mbar_wait(&odone[t], j & 1) && ok;  // P_t(j) consumed
+                    if (!wait(&odone[t], j & 1)) break;  // P_t(j) consumed
                     issue_s(t, jn);
                 }
             }
+            if (!ok) break;
             if (lane == 0) tc_commit(&vempty[s]);
             __syncwarp();
             if (jn < ntiles) {
-                if (!kready) ok = mbar_wait(&kfull[sn], (jn / NS) & 1) && ok;
+                if (!kready && !wait(&kfull[sn], (jn / NS) & 1)) break;
                 if (lane == 0) tc_commit(&kempty[sn]);  // after every S(j+1) above
                 __syncwarp();
             }
         }
-        // every MMA of this CTA has completed before TMEM is released
+        // every MMA of this CTA has completed before TMEM is released (after
+        // a failure: with a short fresh budget)
         if (lane == 0) tc_commit(mma_done);
         __syncwarp();
-        ok = mbar_wait(mma_done, 0) && ok;
+        const bool done = mbar_wait(mma_done, 0, ok ? deadline : drain_deadline());
+        ok = __all_sync(0xffffffffu, ok && done);
     } else {
         // ---- softmax of query tile t: NSPLIT threads per accumulator row,
         // each with SCOL of the row's keys and OCOL of its O columns
@@ -317,17 +345,25 @@ __global__ void __launch_bounds__(C::NT, 1)
         auto xslot = [&](int k, int hh) { return xch + ((k * NQ + t) * NSP + hh) * 128 + r; };
         float m = -INFINITY, l = 0.f;
         for (int j = 0; j < ntl[t]; ++j) {
-            ok = mbar_wait(&sfull[t], j & 1) && ok;
-            tc_fence_after();
+            // after a failed wait this thread issues no further wait and
+            // touches no TMEM, but still meets its partner warp at every named
+            // barrier and arrives on P full, so that no thread is left waiting
+            // on it
             float sv[SCOL];
+            if (wait(&sfull[t], j & 1)) {
+                tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < SCOL / 32; ++q) {
-                float t32[32];
-                tmem_ld32(lane_base + scol + 32 * q, t32);
+                for (int q = 0; q < SCOL / 32; ++q) {
+                    float t32[32];
+                    tmem_ld32(lane_base + scol + 32 * q, t32);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) sv[32 * q + e] = t32[e];
+                    for (int e = 0; e < 32; ++e) sv[32 * q + e] = t32[e];
+                }
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < SCOL; ++e) sv[e] = -INFINITY;
             }
-            tmem_wait_ld();
             // raw scores (the scale is positive, so the max commutes with it);
             // the causal mask only where the tile reaches past this row
             const int kv0 = (jt0 + j) * KT + half * SCOL;
@@ -344,6 +380,10 @@ __global__ void __launch_bounds__(C::NT, 1)
             named_bar_sync(bar_id, 32 * NSP);
 #pragma unroll
             for (int hh = 0; hh < NSP; ++hh) mraw = fmaxf(mraw, *xslot(j & 1, hh));
+            if (!ok) {
+                mbar_arrive(&pfull[t]);
+                continue;
+            }
             const float mt = mraw * sl2;
             const bool rescale = mt > m + kRescaleThreshold;
             float alpha = 1.f;
@@ -396,54 +436,55 @@ __global__ void __launch_bounds__(C::NT, 1)
             l = 0.f;
 #pragma unroll
             for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
-            ok = mbar_wait(&ofinal[t], 0) && ok;
-            tc_fence_after();
-            const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
-            __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;
-            const float inv = (l > 0.f) ? 1.f / l : 0.f;
-            if (shared) {
-                // split-K piece kz of the row: normalised fp32 output and log2-sum-exp
-                const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;
-                float *wo = a.ws_o + (grow * a.max_parts + kz) * D + half * OCOL;
+            if (wait(&ofinal[t], 0)) {
+                tc_fence_after();
+                const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;
+                const float inv = (l > 0.f) ? 1.f / l : 0.f;
+                if (shared) {
+                    // split-K piece kz of the row: normalised fp32 output and log2-sum-exp
+                    const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;
+                    float *wo = a.ws_o + (grow * a.max_parts + kz) * D + half * OCOL;
 #pragma unroll
-                for (int q = 0; q < OCOL / 32; ++q) {
-                    float o[32];
-                    tmem_ld32(lane_base + ocol + 32 * q, o);
-                    tmem_wait_ld();
-                    if (row_valid) {
+                    for (int q = 0; q < OCOL / 32; ++q) {
+                        float o[32];
+                        tmem_ld32(lane_base + ocol + 32 * q, o);
+                        tmem_wait_ld();
+                        if (row_valid) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4 *>(wo + 32 * q + e) =
-                                make_float4(o[e] * inv * vs, o[e + 1] * inv * vs, o[e + 2] * inv * vs,
-                                            o[e + 3] * inv * vs);
+                            for (int e = 0; e < 32; e += 4)
+                                *reinterpret_cast<float4 *>(wo + 32 * q + e) =
+                                    make_float4(o[e] * inv * vs, o[e + 1] * inv * vs, o[e + 2] * inv * vs,
+                                                o[e + 3] * inv * vs);
+                        }
                     }
-                }
-                if (row_valid && half == 0) a.ws_lse[grow * a.max_parts + kz] = (l > 0.f) ? m + lg2(l) : -INFINITY;
-            } else {
+                    if (row_valid && half == 0) a.ws_lse[grow * a.max_parts + kz] = (l > 0.f) ? m + lg2(l) : -INFINITY;
+                } else {
 #pragma unroll
-                for (int q = 0; q < OCOL / 32; ++q) {
-                    float o[32];
-                    tmem_ld32(lane_base + ocol + 32 * q, o);
-                    tmem_wait_ld();
-                    if (row_valid) {
+                    for (int q = 0; q < OCOL / 32; ++q) {
+                        float o[32];
+                        tmem_ld32(lane_base + ocol + 32 * q, o);
+                        tmem_wait_ld();
+                        if (row_valid) {
 #pragma unroll
-                        for (int e = 0; e < 32; e += 8) {
-                            uint32_t wds[4];
+                            for (int e = 0; e < 32; e += 8) {
+                                uint32_t wds[4];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const __nv_bfloat162 bb =
-                                    __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
-                                wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
+                                for (int u = 0; u < 4; ++u) {
+                                    const __nv_bfloat162 bb =
+                                        __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
+                                    wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
+                                }
+                                *reinterpret_cast<uint4 *>(dst + 32 * q + e) =
+                                    make_uint4(wds[0], wds[1], wds[2], wds[3]);
                             }
-                            *reinterpret_cast<uint4 *>(dst + 32 * q + e) =
-                                make_uint4(wds[0], wds[1], wds[2], wds[3]);
                         }
                     }
                 }
-            }
+            }  // O final
         }
     }
-    if (!ok) flag_error(a.err, PA_DEVERR_TIMEOUT);
+    if (!ok && lane == 0) flag_error(a.err, PA_DEVERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (w == C::W_MMA) {

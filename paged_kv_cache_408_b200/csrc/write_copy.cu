@@ -100,7 +100,8 @@ cudaError_t launch_write_kv(const WriteArgs &a, cudaStream_t st) {
     if (n_chunks == 0) return cudaSuccess;
     const int threads = 256;
     int64_t blocks = (n_chunks + threads - 1) / threads;
-    if (blocks > 148 * 64) blocks = 148 * 64;
+    const int64_t cap = (int64_t)sm_count() * 8;  // 8 resident CTAs of 256 threads per SM, grid-stride beyond
+    if (blocks > cap) blocks = cap;
     return launch_pdl(a.fp8 ? write_kv_kernel<true> : write_kv_kernel<false>, dim3((unsigned)blocks), dim3(threads),
                       0, st, (const uint4 *)a.k, (const uint4 *)a.v, a.slots, n_chunks, a.Hkv, a.D, a.num_blocks,
                       a.k_cache, a.v_cache, a.k_scale, a.v_scale, a.err);

@@ -144,3 +144,24 @@ def test_cascade_workspace_size():
     assert cascade_ws(256, 64, 160, 161)[0] == -1
     assert cascade_ws(256, 64, 160, -1)[0] == -1
     assert cascade_ws(256, 64, 160, 0)[1] >= ops.decode_workspace_size(256, 64, 128, 160)
+
+
+def test_block_table_width_is_bounded():
+    """Tables wider than PA_MAX_BLOCKS_PER_SEQ (2^24 entries) are rejected on
+    the host by every entry point that takes one, before any size arithmetic
+    could overflow; the largest accepted width still sizes its workspace."""
+    L = ops.lib()
+    big = (1 << 24) + 1
+    out = C.c_size_t(0)
+    assert L.pa_decode_workspace_size(4, 32, 128, big, 0, C.byref(out)) == -1
+    assert L.pa_decode_workspace_size(4, 32, 128, 1 << 24, 0, C.byref(out)) == 0
+    assert out.value >= 4 * 32 * ((1 << 24) // 16) * 128 * 4
+    assert L.pa_decode_workspace_size(1, 1, 128, 1 << 24, 16, C.byref(out)) == 0  # 2^24 partitions, no wrap
+    assert call_decode(desc(), maxb=big) == -1
+    assert call_decode(desc(), maxb=(1 << 31) - 1) == -1
+    assert call_cascade(desc(), maxb=big, pb=1) == -1
+    assert cascade_ws(4, 32, big, 1)[0] == -1
+    assert L.pa_prefill_chunk(FAKE, FAKE, FAKE, FAKE, FAKE, 2, big, 32, 64, 100, FAKE, FAKE, 0.1, None, None,
+                              C.byref(desc()), None) == -1
+    assert L.pa_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, big, 32, 0.1, None, None, 0,
+                               C.byref(desc()), None) == -1

@@ -152,3 +152,212 @@ def test_a_skipped_o_done_wait_is_caught():
 
 def test_issuing_s_without_the_o_done_wait_is_caught():
     assert explore([5, 6], 2, seeds=200, no_odone_wait=True) is not None
+
+
+# ------------------------------------------------------------------------
+# Giving up after a lost transaction.  Every wait of a launch shares one
+# deadline; in the kernel a role evaluates `ok && mbar_wait(...)`, so after
+# its first failed wait it issues no further wait of the protocol.  The
+# loader and the MMA warp then stop issuing and drain what they have in
+# flight (a short fresh budget); the two softmax warps that share a row
+# keep meeting at their named barrier (which has no deadline) and keep
+# arriving on P full, so neither is left waiting on the other.
+#
+# The model below drops one asynchronous completion at random (a copy or an
+# MMA commit that never arrives).  When no actor can progress, the clock
+# passes the deadline and every blocked wait fails; before that, a blocked
+# wait may also fail on its own now and then (its thread's deadline passed
+# just before a slow completion arrived), so partners can fail at different
+# points of the protocol.  Checked: every actor
+# finishes (no thread stranded at a named barrier), and no actor issues a
+# protocol wait after its first failed one.
+
+def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_failure=False):
+    nq, ntiles = len(ntl), max(ntl)
+    for seed in range(seeds):
+        rnd = random.Random(1000 + seed)
+        ring = {k: [Barrier(f"{k}{i}") for i in range(nslot)] for k in ("kfull", "kempty", "vfull", "vempty")}
+        tile = {k: [Barrier(f"{k}{t}", 2 if k == "pfull" else 1) for t in range(nq)]
+                for k in ("sfull", "pfull", "odone", "ofinal")}
+        mma_done = Barrier("mma_done")
+        pending = []
+        drop_at = rnd.randrange(1, 4 * ntiles * (nq + 2) + 2)
+        sent = [0]
+
+        def post(bar):
+            sent[0] += 1
+            if sent[0] != drop_at:  # the dropped completion never arrives
+                pending.append(bar)
+
+        def wait(bar, phase, ok):
+            """Protocol wait as the kernel issues it: skipped once ok is false."""
+            if ok or wait_after_failure:
+                r = yield ("wait", bar, phase)
+                return ok and r
+            return False
+
+        def loader():
+            ok, issued = True, {"k": 0, "v": 0}
+            for j in range(ntiles):
+                if not ok:
+                    break
+                s, use = j % nslot, j // nslot
+                for kind in ("k", "v"):
+                    if use:
+                        ok = yield from wait(ring[kind + "empty"][s], use - 1, ok)
+                        if not ok:
+                            break
+                    issued[kind] = j + 1
+                    post(ring[kind + "full"][s])
+            if not ok:
+                for kind in ("k", "v"):
+                    for sl in range(nslot):
+                        if issued[kind] > sl:
+                            yield ("drain", ring[kind + "full"][sl], (issued[kind] - 1 - sl) // nslot)
+
+        def mma():
+            ok = True
+            if ntiles:
+                ok = yield from wait(ring["kfull"][0], 0, ok)
+                if ok:
+                    for t in range(nq):
+                        if ntl[t]:
+                            post(tile["sfull"][t])
+                    post(ring["kempty"][0])
+            for j in range(ntiles):
+                if not ok:
+                    break
+                s, jn = j % nslot, j + 1
+                ok = yield from wait(ring["vfull"][s], j // nslot, ok)
+                if not ok:
+                    break
+                kready = False
+                for t in range(nq):
+                    if j < ntl[t]:
+                        ok = yield from wait(tile["pfull"][t], j, ok)
+                        if not ok:
+                            break
+                        post(tile["odone"][t])
+                        if j == ntl[t] - 1:
+                            post(tile["ofinal"][t])
+                    if jn < ntl[t]:
+                        if not kready:
+                            ok = yield from wait(ring["kfull"][jn % nslot], jn // nslot, ok)
+                            if not ok:
+                                break
+                            kready = True
+                        ok = yield from wait(tile["odone"][t], j, ok)
+                        if not ok:
+                            break
+                        post(tile["sfull"][t])
+                if not ok:
+                    break
+                post(ring["vempty"][s])
+                if jn < ntiles:
+                    if not kready:
+                        ok = yield from wait(ring["kfull"][jn % nslot], jn // nslot, ok)
+                        if not ok:
+                            break
+                    post(ring["kempty"][jn % nslot])
+            post(mma_done)
+            yield ("wait" if ok else "drain", mma_done, 0)
+
+        def softmax(t, half):
+            ok = True
+            for j in range(ntl[t]):
+                ok = yield from wait(tile["sfull"][t], j, ok)
+                if not ok and break_softmax_loop:
+                    break
+                yield ("named", t)
+                tile["pfull"][t].arrive()
+            if ntl[t]:
+                yield ("named", t)
+                ok = yield from wait(tile["ofinal"][t], 0, ok)
+
+        actors = {"load": loader(), "mma": mma(),
+                  **{f"softmax{t}.{h}": softmax(t, h) for t in range(nq) for h in range(2)}}
+        state = {k: None for k in actors}   # the event the actor is blocked on
+        reply = {k: None for k in actors}
+        failed = set()
+        named = {}  # t -> actors arrived at the current named barrier
+        expired = False
+        done = set()
+        while len(done) < len(actors):
+            progress = False
+            if pending and rnd.random() < 0.5:
+                pending.pop(0).arrive()
+                progress = True
+            order = list(actors)
+            rnd.shuffle(order)
+            for k in order:
+                if k in done:
+                    continue
+                ev = state[k]
+                if ev is not None:
+                    if ev[0] in ("wait", "drain"):
+                        bar, phase = ev[1], ev[2]
+                        if bar.phase > phase:
+                            reply[k] = True
+                        elif expired or (ev[0] == "wait" and rnd.random() < 0.01):
+                            # past the deadline; or this thread's deadline passed
+                            # just before a slow completion (threads take their
+                            # deadlines at slightly different times)
+                            reply[k] = False
+                            if ev[0] == "wait":
+                                failed.add(k)
+                        else:
+                            continue
+                    elif ev[0] == "named":
+                        if k not in named.get(ev[1], set()):
+                            named.setdefault(ev[1], set()).add(k)
+                        if len(named[ev[1]]) < 2:
+                            continue
+                        reply[k] = None
+                        # the second arriver releases both
+                        other = [a for a in named[ev[1]] if a != k][0]
+                        if state[other] == ev and other != k:
+                            state[other] = ("released",)
+                        named[ev[1]] = set()
+                    elif ev[0] == "released":
+                        reply[k] = None
+                    state[k] = None
+                try:
+                    nxt = actors[k].send(reply[k]) if reply[k] is not None or ev is not None else next(actors[k])
+                except StopIteration:
+                    done.add(k)
+                    progress = True
+                    continue
+                reply[k] = None
+                if nxt[0] == "wait" and k in failed:
+                    return f"seed {seed}: {k} issued a wait after a failed one"
+                state[k] = nxt
+                progress = True
+            if not progress:
+                if pending:
+                    pending.pop(0).arrive()
+                elif not expired:
+                    expired = True  # the clock passes the launch deadline
+                else:
+                    stuck = {k: state[k][:2] if state[k] else None for k in actors if k not in done}
+                    return f"seed {seed}: stranded {stuck}"
+    return None
+
+
+@pytest.mark.parametrize("ntl", [(1, 0), (3, 3), (5, 6), (9, 10)])
+@pytest.mark.parametrize("nslot", [2, 4])
+def test_a_lost_transaction_ends_every_role_without_further_waits(ntl, nslot):
+    assert explore_give_up(list(ntl), nslot, seeds=150) is None
+
+
+def test_softmax_leaving_its_loop_after_a_failure_is_caught():
+    """A softmax warp that stopped at its first failed wait would strand its
+    partner at the named barrier: the model must report it."""
+    found = [explore_give_up([5, 6], ns, seeds=300, break_softmax_loop=True) for ns in (2, 4)]
+    assert any(f and "stranded" in f for f in found), found
+
+
+def test_waiting_again_after_a_failure_is_caught():
+    """Evaluating the wait before the ok flag (waits issued after a failure)
+    must be reported."""
+    found = [explore_give_up([5, 6], ns, seeds=300, wait_after_failure=True) for ns in (2, 4)]
+    assert any(f and "after a failed one" in f for f in found), found
