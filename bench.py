@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0       # B200 HBM3e peak as specified (about 8 TB/s)
 
 METRIC = "paged decode KV-read GB/s (% of B200 HBM peak); seq-steps/s at 64x2K GQA"
 
@@ -191,70 +192,44 @@ TRACES = _Lazy()
 
 
 # ----------------------------------------------------------------- our arm
-class DeviceStep:
-    """One planned step's metadata as device tensors, or (pin=True) packed
-    into one pinned host buffer that to() moves with a single copy."""
-    FIELDS = (("slots", np.int64), ("copies", np.int32), ("tables", np.int32), ("lens", np.int32),
-              ("p_cu", np.int32), ("p_prefix", np.int32), ("p_tables", np.int32))
-
-    def __init__(self, plan, torch, device, pin=False):
-        arrs = {"copies": plan.copies, "slots": plan.slots, "tables": plan.decode_tables,
-                "lens": plan.decode_lens, "p_cu": plan.prefill_cu, "p_prefix": plan.prefill_prefix,
-                "p_tables": plan.prefill_tables}
-        self.plan = plan
-        self.packed = None
-        if pin:
-            # one byte buffer, every field at a 16-byte aligned offset
-            self.layout, off = [], 0
-            for k, dt in self.FIELDS:
-                a = np.ascontiguousarray(arrs[k], dt)
-                self.layout.append((k, dt, off, a.shape))
-                off += (a.nbytes + 15) // 16 * 16
-            host = np.zeros(max(off, 16), np.uint8)
-            for k, dt, o, shape in self.layout:
-                a = np.ascontiguousarray(arrs[k], dt)
-                host[o:o + a.nbytes] = a.view(np.uint8).reshape(-1)
-            self.packed = torch.from_numpy(host).pin_memory()
-        else:
-            for k, dt in self.FIELDS:
-                setattr(self, k, torch.from_numpy(np.ascontiguousarray(arrs[k], dt)).to(device))
-        self.T = len(plan.slots)
-        self.B = plan.num_decode
-        self.nchunks = len(plan.prefill_ids)
-        self.pb = 0  # shared prefix blocks attended by cascade decode (0: plain decode)
-
-    def to(self, device, non_blocking=True):
-        """Device copy of a packed step: one host-to-device copy, then views."""
-        import torch
-        d = object.__new__(DeviceStep)
-        d.__dict__.update(self.__dict__)
-        buf = self.packed.to(device, non_blocking=non_blocking)
-        tdt = {np.int32: torch.int32, np.int64: torch.int64}
-        for k, dt, o, shape in self.layout:
-            n = int(np.prod(shape)) * np.dtype(dt).itemsize
-            setattr(d, k, buf[o:o + n].view(tdt[dt]).view(shape))
-        d.packed = None
-        return d
-
-    def nbytes(self):
-        if self.packed is not None:
-            return self.packed.numel()
-        return sum(getattr(self, k).numel() * getattr(self, k).element_size() for k, _ in self.FIELDS)
+from paged_kv_cache_408_b200.executor import DeviceStep  # noqa: E402  (re-exported for the host tests)
 
 
-def run_ours(args, rank, world, device):
+def prefill_flops(cu_q, prefix_lens, Hq, D):
+    """Algorithmic FLOPs of causal chunked prefill: per chunk of C queries over
+    a prefix of P keys, C*P + C(C+1)/2 query-key pairs, 4*D flops per pair
+    (q.k and p.v), for every query head."""
+    C = np.diff(np.asarray(cu_q, np.int64))
+    P = np.asarray(prefix_lens, np.int64)
+    return int((Hq * 4 * D * (C * P + C * (C + 1) // 2)).sum())
+
+
+def run_ours(args, rank, world, device, workload=None, legs_only=False):
+    """Drive a synthetic trace through the scheduler and the kernels.
+
+    Every step's plan is made on the host first (timed separately); then
+    warm-up steps, then the timed steps, each one programmatic launch chain
+    copy_blocks -> write_kv -> decode (+ merge) [-> prefill], bracketed by
+    CUDA events with the L2 flushed in between (outside the events).  Then
+    the same steps again with only the decode call timed (its roofline), the
+    prefill call (where the trace attends prefill chunks) and, for cascade
+    steps, the suffix stage alone.  legs_only: return only the prefill
+    call's figures (the prefill leg of another workload's run)."""
     import torch
 
-    from paged_kv_cache_408_b200 import ops, traces
+    from paged_kv_cache_408_b200 import ops
+    from paged_kv_cache_408_b200.executor import StepExecutor
 
+    workload = workload or args.workload
     torch.cuda.set_device(device)
-    tr = TRACES[args.workload](args.seed + rank)
+    tr = TRACES[workload](args.seed + rank)
     Hq, Hkv, D, fp8 = tr.Hq, tr.Hkv, tr.D, tr.fp8
     eb = 1 if fp8 else 2
     pool = tr.sched.alloc.num_blocks
     t_plan = time.perf_counter()
     plans = tr.plans(args.warmup + args.steps)
     t_plan = (time.perf_counter() - t_plan) / len(plans)
+    attend_prefill = workload == "mixed"  # elsewhere admitted prompts are written, not attended
 
     g = torch.Generator(device=device).manual_seed(1234 + rank)
     shape = (pool, Hkv, 16, D)
@@ -276,60 +251,43 @@ def run_ours(args, rank, world, device):
     out = torch.empty_like(q)
     pq = torch.randn((max(Pmax_tok, 1), Hq, D), generator=g, device=device).to(torch.bfloat16)
     pout = torch.empty_like(pq)
-    maxb = plans[0].decode_tables.shape[1]
-    pbs = [cascade_blocks(p, args) for p in plans]
-    ws_bytes = max([ops.decode_workspace_size(max(Bmax, 1), Hq, D, maxb, args.partition)] +
-                   [ops.cascade_workspace_size(p.num_decode, Hq, maxb, pb, k_cache) for p, pb in zip(plans, pbs) if pb])
-    ws = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=device)
-    flush = L2Flush(torch, device)
     scale = 1.0 / math.sqrt(D)
-    run_prefill = args.workload == "mixed"
+    ex = StepExecutor(k_cache, v_cache, Hq, scale, k_scale, v_scale, attend_prefill=attend_prefill,
+                      cascade=not args.no_cascade, partition_tokens=args.partition)
+    ex.reserve(plans)
+    flush = L2Flush(torch, device)
 
-    def launch(ds, qq, oo, nk, nv, pqq, poo):
-        n = 0
-        if ds.copies.shape[0]:
-            ops.copy_blocks(k_cache, v_cache, ds.copies)
-            n += 1
-        if ds.T:
-            ops.write_kv(nk[:ds.T], nv[:ds.T], ds.slots, k_cache, v_cache, k_scale, v_scale)
-            n += 1
-        return n
-
-    def decode(ds, qq, oo):
-        if ds.B and ds.pb:
-            ops.decode_cascade(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.tables, ds.lens, scale, ds.pb, ws,
-                               k_scale, v_scale)
-            return 4 if fp8 else 3  # (fp8 widening) + prefix attention + suffix decode + merge
-        if ds.B:
-            ops.decode(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.tables, ds.lens, scale, k_scale, v_scale, ws,
-                       args.partition)
-            return 2  # decode kernel + merge kernel
-        return 0
-
-    def suffix_decode(ds, qq, oo):
-        # the suffix stage of a cascade step on its own: the same keys through
-        # the decode kernel (suffix tables and lengths), for its roofline
-        ops.decode(oo[:ds.B], qq[:ds.B], k_cache, v_cache, ds.sfx_tables, ds.sfx_lens, scale, k_scale, v_scale, ws,
-                   0)
-
-    def prefill(ds, pqq, poo):
-        if run_prefill and ds.nchunks:
-            nt = int(ds.plan.prefill_cu[-1])
-            ops.prefill_chunk(poo[:nt], pqq[:nt], ds.p_cu, ds.p_prefix, ds.p_tables, k_cache, v_cache, scale,
-                              ds.plan.max_chunk)
-            return 1
-        return 0
-
-    dsteps = [DeviceStep(p, torch, device) for p in plans]
-    for ds, pb in zip(dsteps, pbs):
-        ds.pb = pb
-        if pb:
+    dsteps = [DeviceStep(p, torch, device, cascade=not args.no_cascade) for p in plans]
+    for ds in dsteps:
+        if ds.pb:
             st_ = np.full_like(ds.plan.decode_tables, -1)
-            st_[:, :st_.shape[1] - pb] = ds.plan.decode_tables[:, pb:]
+            st_[:, :st_.shape[1] - ds.pb] = ds.plan.decode_tables[:, ds.pb:]
             ds.sfx_tables = torch.from_numpy(st_).to(device)
-            ds.sfx_lens = torch.from_numpy(ds.plan.decode_lens - 16 * pb).to(device)
+            ds.sfx_lens = torch.from_numpy(ds.plan.decode_lens - 16 * ds.pb).to(device)
     torch.cuda.synchronize()
     st = torch.cuda.current_stream()
+
+    def suffix_decode(ds):
+        # the suffix stage of a cascade step on its own: the same keys through
+        # the decode kernel (suffix tables and lengths), for its roofline
+        ops.decode(out[:ds.B], q[:ds.B], k_cache, v_cache, ds.sfx_tables, ds.sfx_lens, scale, k_scale, v_scale,
+                   ex.ws, 0)
+
+    def timed_pass(fn, steps):
+        """fn(ds) for each step, each bracketed by events, L2 flushed in
+        between; a GPU sleep holds the stream while the host enqueues, so the
+        events see device time only."""
+        ev = []
+        torch.cuda._sleep(hold_cycles(len(steps)))
+        for ds in steps:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush()
+            e0.record(st)
+            n = fn(ds)
+            e1.record(st)
+            ev.append((e0, e1, ds, n))
+        torch.cuda.synchronize()
+        return ev
 
     with ClockSampler(torch.cuda.current_device()) as clk:
         # ---- warm-up, with the clock sampler already running: its start-up pause
@@ -337,94 +295,74 @@ def run_ours(args, rank, world, device):
         # timed steps; the warm-up steps flush L2 like the timed ones
         for ds in dsteps[:args.warmup]:
             flush()
-            launch(ds, q, out, new_k, new_v, pq, pout)
-            decode(ds, q, out)
-            prefill(ds, pq, pout)
+            ex.enqueue(ds, q, out, new_k, new_v, pq, pout)
         torch.cuda.synchronize()
         if ops.get_last_device_error() != 0:
             raise RuntimeError("device status word set during warm-up")
-
-        # ---- timed: inputs resident in HBM, L2 flushed between steps (outside the events)
         timed = dsteps[args.warmup:]
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
-        dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in timed]
-        launches = 0
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
         torch.cuda.synchronize()
-        # hold the stream while the host enqueues every timed step, so the
-        # events see device time only (no host launch gaps).  Only the step
-        # is bracketed: an event between two kernels would cut the
-        # programmatic launch chain (write -> decode -> merge -> prefill).
-        torch.cuda._sleep(hold_cycles(len(timed)))
-        for ds, (e0, e1) in zip(timed, ev):
-            flush()
-            e0.record(st)
-            launches += launch(ds, q, out, new_k, new_v, pq, pout)
-            launches += decode(ds, q, out)
-            launches += prefill(ds, pq, pout)
-            e1.record(st)
-        torch.cuda.synchronize()
-        # the decode call alone (its kernel and the merge), same steps and
-        # cache, for the roofline of the dominant kernel
-        torch.cuda._sleep(hold_cycles(len(timed)))
-        for ds, (e0, e1) in zip(timed, dev_ev):
-            flush()
-            e0.record(st)
-            decode(ds, q, out)
-            e1.record(st)
-        torch.cuda.synchronize()
-        sfx_ev = []
-        if any(ds.pb for ds in timed):
-            torch.cuda._sleep(hold_cycles(len(timed)))
-            for ds in timed:
-                if ds.B and ds.pb:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    flush()
-                    e0.record(st)
-                    suffix_decode(ds, q, out)
-                    e1.record(st)
-                    sfx_ev.append((e0, e1, ds))
-            torch.cuda.synchronize()
+        # ---- timed: whole steps (one programmatic launch chain each; an event
+        # inside a step would cut the chain)
+        step_ev = timed_pass(lambda ds: ex.enqueue(ds, q, out, new_k, new_v, pq, pout), timed)
+        # ---- each call alone, same steps and cache, for the kernels' rooflines
+        dec_ev = timed_pass(lambda ds: ex.decode(ds, q, out), [d for d in timed if d.B])
+        pre_ev = timed_pass(lambda ds: ex.prefill(ds, pq, pout), [d for d in timed if d.n_prefill]) \
+            if attend_prefill else []
+        sfx_ev = [] if legs_only else timed_pass(suffix_decode, [d for d in timed if d.B and d.pb])
     if world > 1:
         dist.barrier()
-    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
-    dec_ms = [e0.elapsed_time(e1) for e0, e1 in dev_ev]
+
+    def ms(e):
+        return e[0].elapsed_time(e[1])
+
+    step_ms = [ms(e) for e in step_ev]
+    dec_ms = [ms(e) for e in dec_ev]
     cascade = None
     if sfx_ev:
         n = len(sfx_ev)
-        lens_sfx = [ds.plan.decode_lens - 16 * ds.pb for _, _, ds in sfx_ev]
+        lens_sfx = [e[2].plan.decode_lens - 16 * e[2].pb for e in sfx_ev]
         cascade = {
-            "steps": n, "prefix_blocks": sorted({int(ds.pb) for _, _, ds in sfx_ev}),
-            "call_ms": sum(e0.elapsed_time(e1) for (e0, e1), ds in zip(dev_ev, timed) if ds.B and ds.pb) / n,
-            "suffix_ms": sum(e0.elapsed_time(e1) for e0, e1, _ in sfx_ev) / n,
-            "prefix_flops": sum(4 * D * Hq * ds.B * 16 * ds.pb for _, _, ds in sfx_ev) / n,
+            "steps": n, "prefix_blocks": sorted({int(e[2].pb) for e in sfx_ev}),
+            "call_ms": sum(ms(e) for e in dec_ev if e[2].pb) / n,
+            "suffix_ms": sum(ms(e) for e in sfx_ev) / n,
+            "prefix_flops": sum(4 * D * Hq * e[2].B * 16 * e[2].pb for e in sfx_ev) / n,
             "suffix_flops": sum(decode_alg_flops(x, Hq, D) for x in lens_sfx) / n,
             "suffix_bytes": sum(decode_alg_bytes(x, Hq, Hkv, D, eb) for x in lens_sfx) / n,
-            "unique_bytes": sum(decode_alg_bytes(x, Hq, Hkv, D, eb) + 16 * ds.pb * Hkv * D * 2 * eb
-                                for x, (_, _, ds) in zip(lens_sfx, sfx_ev)) / n,
+            "unique_bytes": sum(decode_alg_bytes(x, Hq, Hkv, D, eb) + 16 * e[2].pb * Hkv * D * 2 * eb
+                                for x, e in zip(lens_sfx, sfx_ev)) / n,
         }
+    prefill = None
+    if pre_ev:
+        pms = [ms(e) for e in pre_ev]
+        pfl = [prefill_flops(e[2].plan.prefill_cu, e[2].plan.prefill_prefix, Hq, D) for e in pre_ev]
+        prefill = {"ms": sum(pms) / len(pms), "flops": sum(pfl) / len(pfl), "steps": len(pms),
+                   "tokens": sum(e[2].n_prefill for e in pre_ev) / len(pre_ev),
+                   "chunks": sum(e[2].nchunks for e in pre_ev) / len(pre_ev), "workload": tr.name,
+                   "clocks": clk.summary()}
+    flags = ops.get_last_device_error()
+    if flags:
+        raise RuntimeError(f"device status word {flags:#x} after the timed steps")
+    if legs_only:
+        return {"prefill": prefill}
+
     tot_ms = sum(step_ms)
     kvb = sum(kv_bytes(ds.plan.decode_lens, Hkv, D, eb) for ds in timed)
     seqsteps = sum(ds.B for ds in timed)
     algb = [decode_alg_bytes(ds.plan.decode_lens, Hq, Hkv, D, eb) for ds in timed if ds.B]
     algf = [decode_alg_flops(ds.plan.decode_lens, Hq, D) for ds in timed if ds.B]
-    flags = ops.get_last_device_error()
-    if flags:
-        raise RuntimeError(f"device status word {flags:#x} after the timed steps")
+    launches = sum(e[3] for e in step_ev)
 
-    # ---- end to end: per-step inputs from pinned host memory, result read back
+    # ---- end to end: per-step inputs from pinned host memory, results read back
     e2e = None
     if not args.no_e2e:
-        hsteps = [DeviceStep(p, torch, device, pin=True) for p in plans[args.warmup:]]
-        for hs, pb in zip(hsteps, pbs[args.warmup:]):
-            hs.pb = pb
-        hq = q.cpu().pin_memory()
-        hk = new_k.cpu().pin_memory()
-        hv = new_v.cpu().pin_memory()
-        hout = torch.empty_like(hq).pin_memory()
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(new_k), torch.empty_like(new_v)
+        hsteps = [DeviceStep(p, torch, device, pin=True, cascade=not args.no_cascade) for p in plans[args.warmup:]]
+        hq, hk, hv = q.cpu().pin_memory(), new_k.cpu().pin_memory(), new_v.cpu().pin_memory()
+        hpq = pq.cpu().pin_memory()
+        hout, hpout = torch.empty_like(hq).pin_memory(), torch.empty_like(hpq).pin_memory()
+        dq, dk, dv, dpq = torch.empty_like(q), torch.empty_like(new_k), torch.empty_like(new_v), torch.empty_like(pq)
         ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in hsteps]
         h2d = d2h = 0
         torch.cuda.synchronize()
@@ -433,166 +371,70 @@ def run_ours(args, rank, world, device):
             e0.record(st)
             ds = hs.to(device)
             nq, nt = hs.B * Hq * D * 2, hs.T * Hkv * D * 2
+            npf = hs.n_prefill * Hq * D * 2 if attend_prefill else 0
             if hs.B:
                 dq[:hs.B].copy_(hq[:hs.B], non_blocking=True)
             if hs.T:
                 dk[:hs.T].copy_(hk[:hs.T], non_blocking=True)
                 dv[:hs.T].copy_(hv[:hs.T], non_blocking=True)
-            launch(ds, dq, out, dk, dv, pq, pout)
-            decode(ds, dq, out)
-            prefill(ds, pq, pout)
+            if npf:
+                dpq[:hs.n_prefill].copy_(hpq[:hs.n_prefill], non_blocking=True)
+            ex.enqueue(ds, dq, out, dk, dv, dpq, pout)
             if hs.B:
                 hout[:hs.B].copy_(out[:hs.B], non_blocking=True)
+            if npf:
+                hpout[:hs.n_prefill].copy_(pout[:hs.n_prefill], non_blocking=True)
             e1.record(st)
-            h2d += hs.nbytes() + nq + 2 * nt
-            d2h += hs.B * Hq * D * 2
+            h2d += hs.nbytes() + nq + 2 * nt + npf
+            d2h += nq + npf
         torch.cuda.synchronize()
         e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
         e2e = {"ms": e2e_ms, "h2d": h2d / len(hsteps), "d2h": d2h / len(hsteps), "kvb": kvb}
 
     return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb, algf=algf,
                 launches=launches, clocks=clk.summary(), e2e=e2e, plan_ms=t_plan * 1e3, tr=tr, plans=plans,
-                cascade=cascade, copies=sum(len(ds.plan.copies) for ds in timed),
+                cascade=cascade, prefill=prefill, copies=sum(len(ds.plan.copies) for ds in timed),
                 k_cache=k_cache, v_cache=v_cache, Hq=Hq, Hkv=Hkv, D=D, eb=eb, fp8=fp8, scale=scale,
                 k_scale=k_scale, v_scale=v_scale, q=q, pool=pool)
 
 
-# ----------------------------------------------------- mixed decode + prefill
-class _StaticStep:
-    """Stand-in for a trace: one fixed step, repeated."""
-
-    def __init__(self, name, Hq, Hkv, D, seqs, pool):
-        from types import SimpleNamespace
-        self.name, self.Hq, self.Hkv, self.D, self.fp8 = name, Hq, Hkv, D, False
-        self.sched = SimpleNamespace(num_preemptions=0, cfg=SimpleNamespace(max_num_seqs=seqs),
-                                     alloc=SimpleNamespace(num_blocks=pool))
-
-
-def prefill_flops(cu_q, prefix_lens, Hq, D):
-    """Algorithmic FLOPs of causal chunked prefill: per chunk of C queries over
-    a prefix of P keys, C*P + C(C+1)/2 query-key pairs, 4*D flops per pair
-    (q.k and p.v), for every query head."""
-    C = np.diff(np.asarray(cu_q, np.int64))
-    P = np.asarray(prefix_lens, np.int64)
-    return int((Hq * 4 * D * (C * P + C * (C + 1) // 2)).sum())
-
-
-def run_mixed(args, rank, world, device):
-    """The mixed step: 192 decode sequences (lognormal lengths, median 1024,
-    capped at 8192) plus 8 prefill chunks of 512 tokens over prefixes uniform
-    in [0, 4096], 32/8 heads, head_dim 128, bf16.  One step = write every new
-    token's K/V, decode, prefill; the same step is repeated."""
-    import torch
-
-    from paged_kv_cache_408_b200 import inputs as I
-    from paged_kv_cache_408_b200 import ops
-
-    torch.cuda.set_device(device)
-    dc, pc = I.mixed_step(args.seed + rank)
-
-    def bf(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
-
-    def it(a, dt):
-        return torch.from_numpy(np.ascontiguousarray(a, dt)).to(device)
-
-    dk, dv = bf(dc.k_cache), bf(dc.v_cache)
-    pk, pv = bf(pc.k_cache), bf(pc.v_cache)
-    dq, pq = bf(dc.q), bf(pc.q)
-    dout, pout = torch.empty_like(dq), torch.empty_like(pq)
-    dnk, dnv, dsl = bf(dc.new_k), bf(dc.new_v), it(dc.slot_mapping, np.int64)
-    pnk, pnv, psl = bf(pc.new_k), bf(pc.new_v), it(pc.slot_mapping, np.int64)
-    dbt, dl = it(dc.block_tables, np.int32), it(dc.seq_lens, np.int32)
-    pcu, ppf, pbt = it(pc.cu_q, np.int32), it(pc.prefix_lens, np.int32), it(pc.block_tables, np.int32)
-    ws = ops.alloc_workspace(dc.B, dc.Hq, dc.D, dc.block_tables.shape[1], args.partition, device=device)
-    flush = L2Flush(torch, device)
-    st = torch.cuda.current_stream()
-
-    def write():
-        ops.write_kv(dnk, dnv, dsl, dk, dv)
-        ops.write_kv(pnk, pnv, psl, pk, pv)
-
-    def decode():
-        ops.decode(dout, dq, dk, dv, dbt, dl, dc.scale, workspace=ws, partition_tokens=args.partition)
-
-    def prefill():
-        ops.prefill_chunk(pout, pq, pcu, ppf, pbt, pk, pv, pc.scale, pc.max_q_len)
-
-    def step():
-        write()
-        decode()
-        prefill()
-        return 5  # two writes, decode + merge, prefill
-
-    def timed(fn, n):
-        """n calls of fn, each bracketed by events, L2 flushed in between."""
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        torch.cuda._sleep(hold_cycles(n))
-        for e0, e1 in ev:
-            flush()
-            e0.record(st)
-            fn()
-            e1.record(st)
-        torch.cuda.synchronize()
-        return [e0.elapsed_time(e1) for e0, e1 in ev]
-
-    # the clock sampler starts before the warm-up: its start-up pause must not
-    # leave the GPU idle right before the timed steps
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for _ in range(args.warmup):
-            flush()
-            step()
-        torch.cuda.synchronize()
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
-        torch.cuda.synchronize()
-        step_ms = timed(step, args.steps)  # the whole step: one programmatic launch chain
-        dec_ms = timed(decode, args.steps)  # then each kernel alone, for its roofline
-        pre_ms = timed(prefill, args.steps)
-    launches = 5 * args.steps
-    if ops.get_last_device_error():
-        raise RuntimeError("device status word set during the mixed step")
-    kvb_step = kv_bytes(dc.seq_lens, dc.Hkv, dc.D, 2)
-    tr = _StaticStep("192 decode seqs (lognormal, median 1024) + 8 prefill chunks x 512 over U[0,4096] "
-                     "prefixes, 32/8 heads, d128, bf16", dc.Hq, dc.Hkv, dc.D, dc.B + len(pc.prefix_lens),
-                     dc.num_blocks + pc.k_cache.shape[0])
-    return dict(tot_ms=sum(step_ms), step_ms=step_ms, dec_ms=dec_ms, kvb=kvb_step * args.steps,
-                seqsteps=dc.B * args.steps, algb=[decode_alg_bytes(dc.seq_lens, dc.Hq, dc.Hkv, dc.D, 2)] * args.steps,
-                algf=[decode_alg_flops(dc.seq_lens, dc.Hq, dc.D)] * args.steps,
-                launches=launches, clocks=clk.summary(), e2e=None, plan_ms=0.0, tr=tr, plans=None, fp8=False,
-                prefill={"ms": sum(pre_ms) / len(pre_ms), "flops": prefill_flops(pc.cu_q, pc.prefix_lens, pc.Hq, pc.D),
-                         "tokens": int(pc.cu_q[-1])})
-
-
 # ------------------------------------------------------------ oracle timing
-def oracle_step_time(plan, kc, vc, q, Hq, scale, ks, vs, rows, nthreads):
-    import oracle
-    t0 = time.perf_counter()
-    oracle.decode(q[rows], kc, vc, plan.decode_tables[rows], plan.decode_lens[rows], scale, ks, vs,
-                  nthreads=nthreads)
-    return time.perf_counter() - t0
-
-
-def cpu_baseline_from(plans, kc, vc, qh, Hq, Hkv, D, eb, scale, ks, vs, budget_s=15.0):
-    """Time the fp64 oracle, as it stands, on whole steps of the same trace
-    until about ``budget_s`` seconds of CPU work are done."""
+def oracle_sample(plans, kc, vc, qh, Hq, Hkv, D, eb, scale, ks, vs, per_step_s=2.0, budget_s=None, warmup=0):
+    """Time the fp64 oracle, as it stands, on the decode of the trace's steps:
+    a whole step where that takes at most about ``per_step_s`` on these
+    cores, else the first n sequences of every step, n sized from a probe of
+    the first step so that a step takes about ``per_step_s``.  ``warmup``
+    steps run untimed first; timing stops after ``budget_s`` seconds if given.
+    Both the CPU baseline of our arm and the reference arm use this sample."""
     import oracle
     nthreads = os.cpu_count() or 1
-    done_b = 0
-    secs = 0.0
-    nsteps = 0
-    for p in plans:
-        rows = np.arange(p.num_decode)
-        secs += oracle_step_time(p, kc, vc, qh[:p.num_decode], Hq, scale, ks, vs, rows, nthreads)
-        done_b += kv_bytes(p.decode_lens, Hkv, D, eb)
+
+    def run(p, rows):
+        t0 = time.perf_counter()
+        oracle.decode(qh[rows], kc, vc, p.decode_tables[rows], p.decode_lens[rows], scale, ks, vs,
+                      nthreads=nthreads)
+        return time.perf_counter() - t0
+
+    Bmax = max(p.num_decode for p in plans)
+    probe = plans[0]
+    n0 = max(1, min(8, probe.num_decode))
+    per_row = run(probe, np.arange(n0)) / n0
+    nrows = int(max(1, min(Bmax, per_step_s / max(per_row, 1e-6))))
+    for p in plans[:warmup]:
+        run(p, np.arange(min(nrows, p.num_decode)))
+    secs, kvb, seqsteps, nsteps = 0.0, 0, 0, 0
+    for p in plans[warmup:]:
+        rows = np.arange(min(nrows, p.num_decode))
+        secs += run(p, rows)
+        kvb += kv_bytes(p.decode_lens[rows], Hkv, D, eb)
+        seqsteps += len(rows)
         nsteps += 1
-        if secs >= budget_s:
+        if budget_s is not None and secs >= budget_s:
             break
-    used = oracle.max_threads()
-    return {"value": done_b / secs / 1e9, "unit": "GB/s", "cores": used, "kind": "oracle",
-            "sample": f"{nsteps} whole decode steps of the same trace (fp64 C oracle, OpenMP over sequence x "
-                      f"head), {secs:.1f} s", "seq_steps_per_s": sum(p.num_decode for p in plans[:nsteps]) / secs}
+    what = "whole steps" if nrows >= Bmax else f"the first {nrows} sequences of each step"
+    return {"value": kvb / secs / 1e9, "unit": "GB/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"decode of {nsteps} steps of the same trace, {what} (fp64 C oracle, OpenMP over sequence "
+                      f"x head), {secs:.1f} s", "seq_steps_per_s": seqsteps / secs, "secs": secs, "steps": nsteps}
 
 
 def host_copy(t, torch):
@@ -625,31 +467,16 @@ def run_reference(args, rank, world):
     Bmax = max(p.num_decode for p in plans)
     qh = I.normal_bf16(rng, (Bmax, tr.Hq, tr.D))
     scale = 1.0 / math.sqrt(tr.D)
-    nthreads = os.cpu_count() or 1
-    # bounded sample per step: the first `rows` sequences of each step, sized
-    # so one step takes about 2 s on these cores
-    probe = plans[0]
-    t1 = oracle_step_time(probe, kc, vc, qh, tr.Hq, scale, ks, vs, np.arange(min(8, probe.num_decode)), nthreads)
-    per_seq = t1 / min(8, probe.num_decode)
-    nrows = int(max(1, min(Bmax, 2.0 / max(per_seq, 1e-6))))
-    for p in plans[:args.warmup]:
-        oracle_step_time(p, kc, vc, qh, tr.Hq, scale, ks, vs, np.arange(min(nrows, p.num_decode)), nthreads)
-    secs = 0.0
-    kvb = 0
-    seqsteps = 0
-    for p in plans[args.warmup:]:
-        rows = np.arange(min(nrows, p.num_decode))
-        secs += oracle_step_time(p, kc, vc, qh, tr.Hq, scale, ks, vs, rows, nthreads)
-        kvb += kv_bytes(p.decode_lens[rows], tr.Hkv, tr.D, eb)
-        seqsteps += len(rows)
-    value = kvb / secs / 1e9
+    smp = oracle_sample(plans, kc, vc, qh, tr.Hq, tr.Hkv, tr.D, eb, scale, ks, vs, per_step_s=2.0,
+                        warmup=args.warmup)
+    value, secs = smp["value"], smp["secs"]
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "impl": "reference", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(args, tr),
-            "seq_steps_per_s": seqsteps / secs,
-            "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": oracle.max_threads(),
-                             "sample": f"first {nrows} sequences of each step of the same trace"},
+            "seq_steps_per_s": smp["seq_steps_per_s"],
+            "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": smp["cores"],
+                             "sample": smp["sample"]},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
 
@@ -724,14 +551,24 @@ def cascade_roofline(c, hbm_peak, hbm_kind, apeak, sm_mhz, workload, cuda_core_m
 
 
 def cascade_blocks(plan, args):
-    """Shared prefix blocks a step's decode attends through cascade decode:
-    every row's leading table entries are the same physical blocks (forked
-    sequences), for a batch and prefix large enough to pay for the extra
-    launches; else 0 (plain decode)."""
-    if args.no_cascade:
-        return 0
-    pb = plan.shared_decode_blocks
-    return pb if plan.num_decode >= 8 and pb * 16 >= 256 else 0
+    """Shared prefix blocks a step's decode attends through cascade decode
+    (0: plain decode); see executor.cascade_blocks."""
+    from paged_kv_cache_408_b200.executor import cascade_blocks as cb
+    return cb(plan, not args.no_cascade)
+
+
+def prefill_block(pf):
+    """The prefill call's figures: algorithmic FLOPs over its CUDA-event time,
+    against the measured bf16 GEMM peak (the call is timed alone)."""
+    tfl = pf["flops"] / (pf["ms"] / 1e3) / 1e12
+    bf16_peak, kind = tensor_peak()
+    return {"tflops": tfl, "ms_per_launch": pf["ms"], "flops_per_launch": pf["flops"],
+            "tokens_per_launch": pf["tokens"], "chunks_per_launch": pf["chunks"], "steps": pf["steps"],
+            "workload": pf["workload"], "clocks": pf.get("clocks"),
+            "roofline": {"bound": "tensor", "achieved": tfl, "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": tfl / bf16_peak, "peak_kind": kind, "kernel": "pa_prefill_chunk (prefill_kernel)",
+                         "timing": "the prefill call of every timed step of the mixed trace alone, CUDA events, "
+                                   "L2 flushed before each"}}
 
 
 def main():
@@ -747,6 +584,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cascade", action="store_true", help="plain decode even where rows share prefix blocks")
+    ap.add_argument("--no-prefill-leg", action="store_true",
+                    help="skip timing the mixed trace's chunked prefill after a decode-only workload")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -768,7 +607,15 @@ def main():
         torch.cuda.set_device(device)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
-    r = run_mixed(args, rank, world, device) if args.workload == "mixed" else run_ours(args, rank, world, device)
+    r = run_ours(args, rank, world, device)
+    # a decode-only workload also times chunked prefill: the prefill call of
+    # the mixed trace (the scheduler's chunks over their paged prefixes)
+    leg = None
+    if args.workload != "mixed" and not args.no_prefill_leg:
+        import types
+        largs = types.SimpleNamespace(**vars(args))
+        largs.steps, largs.warmup = min(args.steps, 10), 3
+        leg = run_ours(largs, rank, world, device, workload="mixed", legs_only=True)["prefill"]
 
     tot_s, kvb, seqsteps = aggregate(r["tot_ms"] / 1e3, r["kvb"], r["seqsteps"], world, device)
 
@@ -792,6 +639,8 @@ def main():
         else:
             roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "peak_kind": f"{peak_kind} (copy bandwidth)"}
+        roof["frac_of_spec"] = achieved / SPEC_HBM_GBS
+        roof["spec_peak"] = SPEC_HBM_GBS
         roof.update({"kernel": "pa_decode (decode + merge)",
                      "traffic": profiled_traffic("paged_kv_cache_408_b200/csrc/decode.cu", args.workload),
                      "alg_bytes_per_launch": alg, "alg_flops_per_launch": flops, "ms_per_launch": dec_ms})
@@ -806,6 +655,8 @@ def main():
             "seq_steps_per_s": seqsteps / tot_s,
             "decode_path": "cascade" if r.get("cascade") else "decode",
             "pct_of_hbm_peak": 100.0 * (kvb / tot_s / 1e9) / peak,
+            "pct_of_hbm_spec": 100.0 * (kvb / tot_s / 1e9) / SPEC_HBM_GBS,
+            "hbm_denominators": {"measured_copy_gbs": peak, "measured_kind": peak_kind, "spec_gbs": SPEC_HBM_GBS},
             "roofline": roof,
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
@@ -819,22 +670,20 @@ def main():
             line["e2e"] = {"value": e["kvb"] / (e["ms"] / 1e3) / 1e9, "unit": "GB/s",
                            "h2d_bytes_per_step": int(e["h2d"]), "d2h_bytes_per_step": int(e["d2h"]),
                            "ms_per_step": e["ms"] / args.steps}
-        if r.get("prefill"):
-            pf = r["prefill"]
-            tfl = pf["flops"] / (pf["ms"] / 1e3) / 1e12
-            bf16_peak, kind = tensor_peak()
-            line["prefill"] = {"tflops": tfl, "ms_per_launch": pf["ms"], "flops_per_launch": pf["flops"],
-                               "tokens": pf["tokens"],
-                               "roofline": {"bound": "tensor", "achieved": tfl, "peak": bf16_peak, "unit": "TFLOP/s",
-                                            "frac": tfl / bf16_peak, "peak_kind": kind, "kernel": "pa_prefill_chunk"}}
+        pf = r.get("prefill") or leg
+        if pf:
+            line["prefill"] = prefill_block(pf)
         if world == 1 and not args.no_cpu_baseline and r.get("plans"):
             import torch as _t
             kc, vc = host_copy(r["k_cache"], _t), host_copy(r["v_cache"], _t)
             qh = host_copy(r["q"], _t)
             ks = r["k_scale"].cpu().numpy() if r["k_scale"] is not None else None
             vs = r["v_scale"].cpu().numpy() if r["v_scale"] is not None else None
-            line["cpu_baseline"] = cpu_baseline_from(r["plans"][args.warmup:], kc, vc, qh, r["Hq"], r["Hkv"],
-                                                     r["D"], r["eb"], r["scale"], ks, vs)
+            cb = oracle_sample(r["plans"][args.warmup:], kc, vc, qh, r["Hq"], r["Hkv"], r["D"], r["eb"], r["scale"],
+                               ks, vs, per_step_s=2.0, budget_s=15.0)
+            cb.pop("secs")
+            cb.pop("steps")
+            line["cpu_baseline"] = cb
         print(json.dumps(line), flush=True)
 
     if world > 1:

@@ -274,13 +274,15 @@ def make_prefill_case(seed, chunk_lens, prefix_lens, Hq, Hkv, D, num_blocks=None
 
 def mixed_step(seed=0, n_decode=192, n_chunks=8, chunk=512):
     """192 decode sequences (lognormal lengths, median 1024, sigma 1, capped
-    at 8192) plus 8 prefill chunks of 512 tokens over prefixes uniform in
-    [0, 4096]; 32/8 heads, head_dim 128, bf16.  The decode part and the
-    prefill part share one pool."""
+    at 8192; block tables 512 entries wide, the cap) plus 8 prefill chunks
+    of 512 tokens over prefixes uniform in [0, 4096]; 32/8 heads, head_dim
+    128, bf16.  Returned as two separate cases (each with its own pool); the
+    scheduler-driven mixed trace runs both halves on one pool."""
     rng = np.random.default_rng(20_000 + seed)
     dec_lens = lognormal_lengths(rng, n_decode)
     prefixes = rng.integers(0, 4097, n_chunks).astype(np.int32)
-    dec = make_decode_case(seed, dec_lens, 32, 8, 128, name="mixed: 192 decode seqs", with_write=True)
+    dec = make_decode_case(seed, dec_lens, 32, 8, 128, name="mixed: 192 decode seqs", with_write=True,
+                           max_blocks=blocks_for(8192))
     pre = make_prefill_case(seed + 1, [chunk] * n_chunks, prefixes, 32, 8, 128,
                             name="mixed: 8 chunks x 512 over U[0,4096] prefixes")
     return dec, pre

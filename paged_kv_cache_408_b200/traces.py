@@ -19,9 +19,14 @@ kernels execute; the caller runs them in order.
 * ``long_context``: 16 sequences of 32768 tokens, 32/8 heads, bf16, blocks
   scattered over a 40960-block pool; every step decodes one more token of
   each (split-K over many partitions).
-* ``mixed``: 192 decode sequences with lognormal lengths (median 1024,
-  sigma 1, capped at 8192) plus prompt requests cut into 512-token chunks
-  over token budget 8192.
+* ``mixed``: chunked prefill interleaved with decode under token budget
+  8192.  Step 0 is 192 decode sequences with lognormal lengths (median 1024,
+  sigma 1, capped at 8192) plus 8 prompts in prefill whose next 512-token
+  chunk attends a cached prefix uniform in [0, 4096]; 32/8 heads, head_dim
+  128, bf16.  Decode sequences stop after Geometric(1/256) steps; a prompt
+  that finishes its prefill joins the decode batch; new prompts (U[512, 4608]
+  tokens) arrive so that 8 prompts are always in prefill, each advancing by
+  one chunk of at most 512 tokens per step.
 """
 from __future__ import annotations
 
@@ -123,19 +128,40 @@ def prefix_share_fp8(seed=0, n=256, forks=32, prefix=2048) -> Trace:
     return tr
 
 
-def mixed(seed=0, n_decode=192, chunk=512, n_prompts=8) -> Trace:
+def _keep_prompts_in_prefill(tr: Trace, n_prompts, chunk, p):
+    """New prompts arrive so that n_prompts are in prefill (running or
+    waiting): U[chunk, 4096 + chunk] tokens each, then Geometric(p) decode
+    steps."""
+    busy = sum(1 for s in tr.sched.running if s.in_prefill) + len(tr.sched.waiting)
+    for _ in range(n_prompts - busy):
+        L = int(tr.rng.integers(chunk, 4096 + chunk + 1))
+        tr.sched.add_request(Sequence(tr.new_id(), L, int(tr.rng.geometric(p))))
+
+
+def mixed(seed=0, n_decode=192, chunk=512, n_prompts=8, headroom_steps=48, p=1.0 / 256) -> Trace:
     rng = np.random.default_rng(60_000 + seed)
-    lens = I.lognormal_lengths(rng, n_decode)
-    prompts = rng.integers(0, 4097, n_prompts) + chunk  # prefix U[0,4096] + one chunk to go
-    need = int(sum(blocks_for(int(L)) for L in lens)) + int(sum(blocks_for(int(p)) for p in prompts))
-    pool = int(math.ceil(1.1 * need)) + 1024
+    lens = I.lognormal_lengths(rng, n_decode)        # decode-step lengths (incl. the step's own token)
+    prefixes = rng.integers(0, 4097, n_prompts)      # cached part of each prompt in prefill
+    togo = chunk * rng.integers(1, 5, n_prompts)     # its chunks still to run (1..4 of 512)
+    need = int(sum(blocks_for(int(L)) for L in lens)) + int(sum(blocks_for(int(a + b))
+                                                                 for a, b in zip(prefixes, togo)))
+    # room for the prompts of headroom_steps steps (about n_prompts*chunk tokens a step) on top of 1.1x
+    pool = int(math.ceil(1.1 * need)) + blocks_for(headroom_steps * n_prompts * chunk)
     alloc = BlockAllocator(pool, order=rng.permutation(pool))
-    cfg = SchedulerConfig(max_num_seqs=n_decode + n_prompts, max_num_batched_tokens=8192, max_chunk=chunk,
+    cfg = SchedulerConfig(max_num_seqs=n_decode + 8 * n_prompts, max_num_batched_tokens=8192, max_chunk=chunk,
                           max_blocks_per_seq=blocks_for(8192 + 4096 + chunk))
     sched = Scheduler(alloc, cfg)
-    tr = Trace("192 decode seqs + 512-token prefill chunks, 32/8 heads, d128, bf16", sched, 32, 8, 128, False, rng)
+    tr = Trace(f"{n_decode} decode seqs (lognormal, median 1024, cap 8192) + {n_prompts} prefill chunks x "
+               f"{chunk} over U[0,4096] prefixes, budget 8192, 32/8 heads, d128, bf16", sched, 32, 8, 128, False, rng,
+               before_step=lambda t: _keep_prompts_in_prefill(t, n_prompts, chunk, p))
     for L in lens:
-        sched.restore(tr.new_id(), int(L) - 1, 10 ** 9)
+        sched.restore(tr.new_id(), int(L) - 1, int(rng.geometric(p)))
+    for a, b in zip(prefixes, togo):
+        # a prompt part-way through its prefill: a cached prefix, chunks to go
+        s = Sequence(tr.new_id(), int(a + b), int(rng.geometric(p)), num_cached=int(a), prefill_end=int(a + b))
+        for _ in range(blocks_for(int(a))):
+            s.block_table.append(alloc.alloc())
+        sched.add_running(s)
     tr.info["pool_blocks"] = pool
     return tr
 

@@ -105,18 +105,13 @@ def test_cascade_workspace_reuse_across_batches(cuda_device):
     assert ops.get_last_device_error() == 0
 
 
-def test_cascade_prefix_share_fp8_full_size_sampled(cuda_device):
+def test_cascade_prefix_share_fp8_full_size_every_row(cuda_device):
     """256 sequences over one shared 2048-token prefix (128 blocks) with
-    suffixes in [16, 512], 64/8 heads, fp8: sampled rows against the oracle,
-    and every row against the plain decode kernel's output."""
+    suffixes in [16, 512], 64/8 heads, fp8: every row against the oracle."""
     c = I.prefix_share(0)
     kc, vc = cache_to_device(c)
     got = run_cascade(c, kc, vc, 128)
-    rows = np.random.default_rng(3).choice(c.B, 24, replace=False)
-    assert_attn_close(got[rows], oracle_of(c, rows=rows), "256 x 2048 shared, sampled")
-    from gpu_util import run_decode
-    plain = to_float(run_decode(c, kc, vc))
-    assert_attn_close(got, plain, "cascade vs decode, every row")
+    assert_attn_close(got, oracle_of(c), "256 x 2048 shared")
     assert ops.get_last_device_error() == 0
 
 

@@ -122,34 +122,57 @@ def test_copy_blocks_is_bit_exact(cuda_device, fp8):
 
 
 # ------------------------------------------------- full-size workloads
-def test_batch64_2k_full_size_sampled(cuda_device):
+@pytest.mark.parametrize("part", [0, 512])
+def test_batch64_2k_full_size_every_row(cuda_device, part):
+    """64 sequences x U[1,2048] tokens, 32/8 heads, d128, bf16: the step's
+    write, then every row of the decode against the oracle (balanced split
+    and fixed 512-token partitions)."""
     c = I.batch64_2k(0)
     kc, vc = cache_to_device(c)
     ops.write_kv(dev_bf16(c.new_k), dev_bf16(c.new_v), dev(c.slot_mapping, np.int64), kc, vc)
     kh, vh = c.k_cache.copy(), c.v_cache.copy()
     oracle.write_kv(c.new_k, c.new_v, c.slot_mapping, kh, vh)
     assert np.array_equal(host_bits(kc), kh) and np.array_equal(host_bits(vc), vh)
-    out = to_float(run_decode(c, kc, vc))
-    rows = np.random.default_rng(1).choice(c.B, 12, replace=False)
-    rows = np.union1d(rows, [int(np.argmax(c.seq_lens)), int(np.argmin(c.seq_lens))])
-    assert_attn_close(out[rows], oracle_decode(c, kh, vh, rows=rows), "64 x U[1,2048]")
-
-
-def test_long_context_split_k_sampled(cuda_device):
-    c = I.long_context(0)
-    kc, vc = cache_to_device(c)
-    out = to_float(run_decode(c, kc, vc))
-    rows = np.array([0, 9])
-    assert_attn_close(out[rows], oracle_decode(c, rows=rows), "16 x 32768")
+    out = to_float(run_decode(c, kc, vc, partition_tokens=part))
+    assert_attn_close(out, oracle_decode(c, kh, vh), "64 x U[1,2048]")
     assert ops.get_last_device_error() == 0
 
 
-def test_prefix_share_fp8_sampled(cuda_device):
+def test_long_context_split_k_every_row(cuda_device):
+    """16 sequences x 32768 tokens over a 40960-block pool: split-K with
+    every row merged from many pieces; every row against the oracle."""
+    c = I.long_context(0)
+    kc, vc = cache_to_device(c)
+    out = to_float(run_decode(c, kc, vc))
+    assert_attn_close(out, oracle_decode(c), "16 x 32768")
+    assert ops.get_last_device_error() == 0
+
+
+def test_prefix_share_fp8_every_row(cuda_device):
+    """256 sequences sharing a 2048-token prefix plus U[16,512] suffixes,
+    64/8 heads, fp8: plain decode (tensor-core GQA-8 path), every row."""
     c = I.prefix_share(0)
     kc, vc = cache_to_device(c)
     out = to_float(run_decode(c, kc, vc))
-    rows = np.random.default_rng(2).choice(c.B, 12, replace=False)
-    assert_attn_close(out[rows], oracle_decode(c, rows=rows), "256 seqs, shared 2048 prefix, fp8")
+    assert_attn_close(out, oracle_decode(c), "256 seqs, shared 2048 prefix, fp8")
+    assert ops.get_last_device_error() == 0
+
+
+def test_mixed_step_decode_half_every_row(cuda_device):
+    """The decode half of the mixed step: 192 sequences with lognormal
+    lengths (median 1024, sigma 1, capped at 8192), 32/8 heads, d128, bf16,
+    block tables 512 entries wide (the 8192-token cap); the step's write,
+    then every row against the oracle."""
+    dc, _ = I.mixed_step(0)
+    assert dc.block_tables.shape[1] == 512 and dc.seq_lens.max() <= 8192
+    kc, vc = cache_to_device(dc)
+    ops.write_kv(dev_bf16(dc.new_k), dev_bf16(dc.new_v), dev(dc.slot_mapping, np.int64), kc, vc)
+    kh, vh = dc.k_cache.copy(), dc.v_cache.copy()
+    oracle.write_kv(dc.new_k, dc.new_v, dc.slot_mapping, kh, vh)
+    assert np.array_equal(host_bits(kc), kh) and np.array_equal(host_bits(vc), vh)
+    out = to_float(run_decode(dc, kc, vc))
+    assert_attn_close(out, oracle_decode(dc, kh, vh), "192 lognormal")
+    assert ops.get_last_device_error() == 0
 
 
 # ------------------------------------------------ device-side bounds checks
