@@ -36,8 +36,11 @@
 //    so a tile never waits for the other tile's softmax.
 //  * Softmax applies the causal mask only on tiles that reach past the
 //    row's position, moves the running max only when it grows by more than
-//    8 (log2 units), and computes P with one packed FMA and one MUFU.EX2
-//    per score.
+//    8 (log2 units), and computes P with one packed FMA and one
+//    exponential per score: 5 of every 8 pairs on MUFU (ex2.approx), 3 on
+//    the FMA pipe (fastexp.cuh), so that neither unit sets the pace; the
+//    row sum l adds P as rounded to bf16 for the P.V product, so numerator
+//    and denominator use the same weights.
 //  * Every mbarrier is waited on in phase order and never falls two phases
 //    behind its producer (a parity wait cannot tell phase k from k+2); the
 //    protocol was checked against that rule, and for deadlock, by a
@@ -50,6 +53,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "fastexp.cuh"
 #include "tc.cuh"
 
 namespace pa {
@@ -57,6 +61,11 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
+// Of every 8 pairs of scores a softmax thread exponentiates, kEmuPairs go
+// through the FMA-pipe exponential (fastexp.cuh) and the rest through MUFU:
+// with head_dim 128 MUFU alone needs as many clocks per tile as the two
+// MMAs of a query tile, which would leave the tensor core waiting.
+constexpr int kEmuPairs = 3;
 
 template <int D_, int G_>
 struct PCfg {
@@ -403,10 +412,13 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
                 for (int e = 0; e < 64; e += 2) {
                     const float2 x = ffma2(make_float2(sv[64 * h + e], sv[64 * h + e + 1]), sc2, nb2);
-                    const float p0 = ex2(x.x), p1 = ex2(x.y);
-                    sum2 = fadd2(sum2, make_float2(p0, p1));
-                    const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-                    pk[e / 2] = *reinterpret_cast<const uint32_t *>(&bb);
+                    const float2 pp = ((e / 2) % 8 < kEmuPairs) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(pp.x, pp.y);
+                    const uint32_t wb = *reinterpret_cast<const uint32_t *>(&bb);
+                    pk[e / 2] = wb;
+                    // the normaliser sums the probabilities as rounded for P.V,
+                    // so the output is an exact weighted mean of V rows
+                    sum2 = fadd2(sum2, make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
                 }
                 tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
             }
