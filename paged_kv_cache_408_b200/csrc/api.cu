@@ -213,8 +213,6 @@ int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const i
                      int32_t num_q_heads, int32_t max_q_len, int32_t total_q_tokens, const void *k_cache,
                      const void *v_cache, float scale, const float *k_scale, const float *v_scale,
                      const pa_cache_desc *desc, pa_stream_t stream) {
-    (void)k_scale;
-    (void)v_scale;
     int rc = check_desc(desc);
     if (rc != PA_OK) return rc;
     if (num_chunks < 0 || max_blocks_per_seq <= 0 || max_blocks_per_seq > pa::kMaxBlocksPerSeq ||
@@ -223,13 +221,19 @@ int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const i
     if (num_q_heads % desc->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int G = num_q_heads / desc->num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
-    if (desc->dtype != PA_DTYPE_BF16) return PA_ERR_UNSUPPORTED;
+    const bool fp8 = desc->dtype == PA_DTYPE_FP8_E4M3;
+    if (fp8 && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
     if (num_chunks == 0 || max_q_len == 0 || total_q_tokens == 0) return PA_OK;
     if (!out || !q || !cu_q_lens || !prefix_lens || !block_tables || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_INVALID_ARG;
     pa::PrefillArgs a{out, q, cu_q_lens, prefix_lens, block_tables, num_chunks, max_blocks_per_seq, num_q_heads,
                       desc->num_kv_heads, desc->head_dim, max_q_len, total_q_tokens, desc->num_blocks, k_cache,
                       v_cache, scale, status_word_ptr()};
+    if (fp8) {
+        a.fp8 = true;
+        a.k_scale = k_scale;
+        a.v_scale = v_scale;
+    }
     return from_cuda(pa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 

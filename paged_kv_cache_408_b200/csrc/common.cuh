@@ -115,10 +115,10 @@ PA_DEVICE void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes, ui
         : "memory");
 }
 
-// Named barrier `id` (1..15) over `nthreads` threads (a multiple of 32).
 // Fetch the 128-byte line holding p into L2 (no register result, no wait).
 PA_DEVICE void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
+// Named barrier `id` (1..15) over `nthreads` threads (a multiple of 32).
 PA_DEVICE void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -181,6 +181,13 @@ PA_DEVICE float2 bf16x2_to_float2(uint32_t w) {
 PA_DEVICE float2 e4m3x2_to_float2(uint16_t w) {
     __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
     return __half22float2(*reinterpret_cast<__half2 *>(&h));
+}
+
+// Two E4M3 codes (low byte first) -> f16x2 (low element first), exact:
+// every E4M3 value is an f16 normal number or zero.
+PA_DEVICE uint32_t e4m3x2_to_h2(uint32_t w16) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w16 & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
 }
 
 // Device status word (PA_DEVERR_* bits).

@@ -475,12 +475,6 @@ PA_DEVICE uint32_t movmatrix_trans(uint32_t x) {
     return y;
 }
 
-// Two E4M3 codes (low byte first) -> f16x2, exact.
-PA_DEVICE uint32_t e4m3x2_to_h2(uint32_t w16) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w16 & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
 PA_DEVICE uint32_t f2_to_h2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);

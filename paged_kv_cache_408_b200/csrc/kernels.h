@@ -75,6 +75,9 @@ struct PrefillArgs {
     float *ws_o, *ws_lse;
     int max_parts;
     int key_splits;
+    // E4M3 cache (k_scale / v_scale required): K/V tiles are widened to f16
+    // on the way into shared memory and the MMAs take f16 operands
+    bool fp8;
 };
 
 cudaError_t launch_write_kv(const WriteArgs &a, cudaStream_t st);

@@ -67,9 +67,10 @@ constexpr float kRescaleThreshold = 8.0f;
 // MMAs of a query tile, which would leave the tensor core waiting.
 constexpr int kEmuPairs = 3;
 
-template <int D_, int G_>
+template <int D_, int G_, bool FP8_>
 struct PCfg {
     static constexpr int D = D_, G = G_;
+    static constexpr bool FP8 = FP8_;             // E4M3 cache: f16 operands, K/V widened by converter warps
     static constexpr int M = 128;                 // accumulator rows of a query tile
     static constexpr int QPOS = M / G;            // query positions per query tile
     static constexpr int NQ = 2;                  // query tiles per CTA
@@ -79,20 +80,35 @@ struct PCfg {
     static constexpr int KATOM = KT * 128;        // bytes of one atom column of a K/V tile
     static constexpr int QTILE = NATOM * QATOM;
     static constexpr int KTILE = NATOM * KATOM;
-    static constexpr int NSLOT = (D == 128) ? 2 : 4;  // K and V ring depth
+    static constexpr int NSLOT = (D == 128 || FP8) ? 2 : 4;  // K and V ring depth
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + NQ * QTILE;
     static constexpr int OFF_V = OFF_K + NSLOT * KTILE;
     static constexpr int NSPLIT = 2;              // softmax threads per accumulator row
     static constexpr int SCOL = KT / NSPLIT;      // S columns (keys) per softmax thread
     static constexpr int OCOL = D / NSPLIT;       // O columns per softmax thread
-    static constexpr int OFF_X = OFF_V + NSLOT * KTILE;  // row max / sum exchange of a row's threads
+    // E4M3 cache: a K or V tile arrives as KT rows of D codes (row-major, by
+    // TMA) in a staging area and is widened there into its f16 slot.  With
+    // head_dim 128 the staging area is the slot's own second atom column: the
+    // thread that widens row i writes that column's row i exactly over row i
+    // of the codes, which it has read first.  With head_dim 64 the slot has
+    // one atom column, so the codes get a ring of their own.
+    static constexpr int STG_BYTES = KT * D;      // one tile of codes
+    static constexpr bool STG_IN_PLACE = FP8 && D == 128;
+    static constexpr int OFF_STG = OFF_V + NSLOT * KTILE;
+    static constexpr int STG_RING = (FP8 && !STG_IN_PLACE) ? 2 * NSLOT * STG_BYTES : 0;
+    static constexpr int OFF_X = OFF_STG + STG_RING;  // row max / sum exchange of a row's threads
     static constexpr int OFF_BAR = OFF_X + 3 * NQ * NSPLIT * 128 * 4;
-    static constexpr int NBAR = 4 * NSLOT + 4 * NQ + 1;  // K/V full+empty; S full, P full, O done, O final; end
+    // K/V full+empty; S full, P full, O done, O final; end; (E4M3) K/V codes loaded
+    static constexpr int NBAR = 4 * NSLOT + 4 * NQ + 1 + (FP8 ? 2 * NSLOT : 0);
     static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // barriers, TMEM slot, alignment slack
     static constexpr int NSMW = NQ * 4 * NSPLIT;  // softmax warps
-    static constexpr int W_LOAD = NSMW, W_MMA = NSMW + 1;
-    static constexpr int NT = (NSMW + 2) * 32;
+    // loader warps: one TMA warp (bf16 cache), or four converter warps that
+    // widen E4M3 K/V rows into the operand tiles (one key row per thread)
+    static constexpr int NLOAD = FP8 ? 2 : 1;
+    static constexpr int W_LOAD = NSMW, W_MMA = NSMW + NLOAD;
+    static constexpr int NT = (NSMW + NLOAD + 1) * 32;
+    static constexpr uint32_t FULL_ARRIVALS = FP8 ? NLOAD * 32 : 1;  // arrivals that fill a K or V slot
     // TMEM columns: S_t (and P_t in its first KT/2 columns) at t * KT; O_t at COL_O + t * D
     static constexpr uint32_t COL_O = NQ * KT;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -116,6 +132,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     uint64_t *kfull = bars, *kempty = bars + NS, *vfull = bars + 2 * NS, *vempty = bars + 3 * NS;
     uint64_t *sfull = bars + 4 * NS, *pfull = sfull + NQ, *odone = pfull + NQ, *ofinal = odone + NQ;
     uint64_t *mma_done = ofinal + NQ;
+    uint64_t *kload = mma_done + 1, *vload = kload + NS;  // E4M3: the codes of a tile have landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
     float *xch = reinterpret_cast<float *>(smem + C::OFF_X);  // [3][NQ][NSPLIT][128]: max (2 parities), sum
 
@@ -160,7 +177,8 @@ __global__ void __launch_bounds__(C::NT, 1)
 
     if (w == C::W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 4 * NS; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 4 * NS; ++i)  // full barriers: [0, NS) and [2NS, 3NS)
+            mbar_init(&bars[i], (i < NS || (i >= 2 * NS && i < 3 * NS)) ? C::FULL_ARRIVALS : 1);
         for (int t = 0; t < NQ; ++t) {
             mbar_init(&sfull[t], 1);
             mbar_init(&pfull[t], 128 * C::NSPLIT);
@@ -168,9 +186,16 @@ __global__ void __launch_bounds__(C::NT, 1)
             mbar_init(&ofinal[t], 1);
         }
         mbar_init(mma_done, 1);
+        if constexpr (C::FP8)
+            for (int i = 0; i < 2 * NS; ++i) mbar_init(&kload[i], 1);
         fence_mbar_init();
     }
-    // ---- query tiles: row r of tile t = (position r / G, head r % G), 128-byte swizzle
+    // ---- query tiles: row r of tile t = (position r / G, head r % G), 128-byte swizzle.
+    // With an E4M3 cache the operands are f16: each row is scaled by a power
+    // of two 2^qexp that puts its largest magnitude in [2^14, 2^15) (exact for
+    // every bf16 value in f16's normal range), and 2^-qexp is folded into the
+    // row's softmax scale.
+    int qexp = 0;
     if (w < C::NSMW) {
         const int t = w / (4 * C::NSPLIT), half = (w / 4) % C::NSPLIT, r = (w % 4) * 32 + lane;
         const int ip = i0 + t * C::QPOS + r / G;
@@ -178,11 +203,46 @@ __global__ void __launch_bounds__(C::NT, 1)
         const __nv_bfloat16 *src =
             static_cast<const __nv_bfloat16 *>(a.q) + ((size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G) * D;
         uint8_t *dst = sQ + t * C::QTILE + r * 128;
+        constexpr int NCH = D / 8 / C::NSPLIT;  // 16-byte chunks of the row per thread
+        uint4 v[NCH];
 #pragma unroll
-        for (int ch = half; ch < D / 8; ch += C::NSPLIT) {
-            const uint4 v = valid ? *reinterpret_cast<const uint4 *>(src + ch * 8) : make_uint4(0, 0, 0, 0);
-            const int at = ch / 8, cc = ch % 8;
-            *reinterpret_cast<uint4 *>(dst + at * C::QATOM + ((cc ^ (r & 7)) * 16)) = v;
+        for (int k = 0; k < NCH; ++k)
+            v[k] = valid ? *reinterpret_cast<const uint4 *>(src + (half + k * C::NSPLIT) * 8) : make_uint4(0, 0, 0, 0);
+        if constexpr (C::FP8) {
+            float amax = 0.f;
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) {
+                const uint32_t ws[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = bf16x2_to_float2(ws[e]);
+                    amax = fmax3(amax, fabsf(f.x), fabsf(f.y));
+                }
+            }
+            float *xq = xch + ((2 * NQ + t) * C::NSPLIT) * 128 + r;  // the sum slots, free until the epilogue
+            xq[half * 128] = amax;
+            named_bar_sync(1 + t * 4 + (w % 4), 32 * C::NSPLIT);
+#pragma unroll
+            for (int hh = 0; hh < C::NSPLIT; ++hh) amax = fmaxf(amax, xq[hh * 128]);
+            if (amax > 0.f) qexp = min(max(14 - ((int)((__float_as_uint(amax) >> 23) & 0xff) - 127), -60), 60);
+            const float qs = __uint_as_float((uint32_t)(127 + qexp) << 23);
+#pragma unroll
+            for (int k = 0; k < NCH; ++k) {
+                const uint32_t ws[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+                uint32_t hw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = bf16x2_to_float2(ws[e]);
+                    const __half2 h = __floats2half2_rn(f.x * qs, f.y * qs);
+                    hw[e] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+                v[k] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+            const int ch = half + k * C::NSPLIT, at = ch / 8, cc = ch % 8;
+            *reinterpret_cast<uint4 *>(dst + at * C::QATOM + ((cc ^ (r & 7)) * 16)) = v[k];
         }
     }
     fence_proxy_async_smem();
@@ -204,7 +264,105 @@ __global__ void __launch_bounds__(C::NT, 1)
         return ok;
     };
 
-    if (w == C::W_LOAD) {
+    if (C::FP8 && w >= C::W_LOAD && w < C::W_MMA) {
+        // ---- E4M3 cache: the first loader warp gathers each K and V tile's
+        // codes (8 paged blocks, 2-D TMA boxes of 16 rows x D bytes, no
+        // multicast) into the tile's staging area; both loader warps widen
+        // the staged rows exactly to f16 into the 128-byte swizzled operand
+        // layout (thread ct: rows ct and ct + 64), zero the rows past the
+        // sequence end, fence the stores for the tensor core and arrive on
+        // the slot's full barrier.  A slot is refilled once the MMAs reading
+        // its previous tile have completed (its empty barrier).
+        constexpr int BPT = KT / 16;  // blocks per tile
+        const int ct = tid - C::W_LOAD * 32;
+        const bool issuer = w == C::W_LOAD;
+        int win0 = jt0 * BPT, went = issuer ? bt[min(win0 + lane, nalloc - 1)] : 0;
+        auto stage = [&](int s, int kv) -> uint8_t * {
+            if constexpr (C::STG_IN_PLACE) return (kv ? sV : sK) + s * C::KTILE + C::KATOM;
+            return smem + C::OFF_STG + (2 * s + kv) * C::STG_BYTES;
+        };
+        auto issue = [&](int j, int kv) {  // issuer warp: TMA of tile j's codes of K (kv 0) or V
+            const int s = j % NS, jb = (jt0 + j) * BPT;
+            if (jb + BPT > win0 + 32) {
+                win0 = jb;
+                went = bt[min(win0 + lane, nalloc - 1)];
+            }
+            int phys = __shfl_sync(0xffffffffu, went, (min(jb + lane % BPT, nalloc - 1) - win0) & 31);
+            if (lane < BPT && (phys < 0 || phys >= a.num_blocks)) {
+                flag_error(a.err, PA_DEVERR_BAD_BLOCK);
+                phys = 0;
+            }
+            uint64_t *ld = kv ? &vload[s] : &kload[s];
+            if (lane == 0) mbar_arrive_expect_tx(ld, C::STG_BYTES);
+            __syncwarp();
+            if (lane < BPT) tma_load_2d(stage(s, kv) + lane * 16 * D, kv ? &tmV : &tmK, 0, (phys * a.Hkv + kvh) * 16, ld);
+            __syncwarp();
+        };
+        auto widen = [&](int j, int kv) {  // both warps: tile j's staged codes -> f16 operand slot
+            const int s = j % NS;
+            if (!wait(kv ? &vload[s] : &kload[s], (j / NS) & 1)) return false;
+            uint8_t *tile = (kv ? sV : sK) + s * C::KTILE;
+            const uint8_t *codes = stage(s, kv);
+#pragma unroll
+            for (int h = 0; h < KT / 64; ++h) {
+                const int i = ct + 64 * h;                      // key row of the tile
+                const bool live = (jt0 + j) * KT + i < L;
+                uint4 src[D / 16];
+#pragma unroll
+                for (int u = 0; u < D / 16; ++u)
+                    src[u] = live ? *reinterpret_cast<const uint4 *>(codes + i * D + 16 * u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < D / 16; ++u) {
+                    const uint32_t ws[4] = {src[u].x, src[u].y, src[u].z, src[u].w};
+                    uint32_t hv[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hv[2 * e] = e4m3x2_to_h2(ws[e]);
+                        hv[2 * e + 1] = e4m3x2_to_h2(ws[e] >> 16);
+                    }
+#pragma unroll
+                    for (int hc = 0; hc < 2; ++hc) {  // f16 chunk 2u + hc: 8 elements
+                        const int ch = 2 * u + hc, at = ch / 8, cc = ch % 8;
+                        *reinterpret_cast<uint4 *>(tile + at * C::KATOM + i * 128 + ((cc ^ (i & 7)) * 16)) =
+                            make_uint4(hv[4 * hc], hv[4 * hc + 1], hv[4 * hc + 2], hv[4 * hc + 3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(kv ? &vfull[s] : &kfull[s]);
+            return true;
+        };
+        int kissued = 0, vissued = 0;  // tiles whose codes were requested
+        if (issuer)
+            for (int j = 0; j < min(NS, ntiles); ++j) {
+                issue(j, 0);
+                issue(j, 1);
+                kissued = vissued = j + 1;
+            }
+        for (int j = 0; j < ntiles && ok; ++j) {
+            if (!widen(j, 0) || !widen(j, 1)) break;
+            // refill the slot of tile j-1 with tile j-1+NS once its MMAs are done
+            const int jr = j - 1 + NS;
+            if (issuer && j >= 1 && jr < ntiles) {
+                if (!wait(&kempty[(j - 1) % NS], ((j - 1) / NS) & 1)) break;
+                issue(jr, 0);
+                kissued = jr + 1;
+                if (!wait(&vempty[(j - 1) % NS], ((j - 1) / NS) & 1)) break;
+                issue(jr, 1);
+                vissued = jr + 1;
+            }
+        }
+        if (!ok && issuer) {
+            // each slot has at most one fill of codes in flight: wait for the
+            // last one of every slot, with a short fresh budget
+            const uint64_t dd = drain_deadline();
+            for (int sl = 0; sl < NS; ++sl) {
+                if (kissued > sl) mbar_wait(&kload[sl], ((kissued - 1 - sl) / NS) & 1, dd);
+                if (vissued > sl) mbar_wait(&vload[sl], ((vissued - 1 - sl) / NS) & 1, dd);
+            }
+            __syncwarp();
+        }
+    } else if (!C::FP8 && w == C::W_LOAD) {
         // ---- producer: K tile j, then V tile j, into ring slot j % NS.  The
         // warp keeps a window of 32 block-table entries in registers (lane l
         // holds entry win0 + l), refilled every 32/BPT tiles, so a tile's
@@ -259,8 +417,8 @@ __global__ void __launch_bounds__(C::NT, 1)
         // as soon as that P.V has completed (S_t(j+1) overwrites P_t).  Tile
         // 0's next scores never wait for tile 1's softmax, and tile 1 stays
         // half a step behind tile 0, so the two softmaxes use MUFU in turns.
-        constexpr uint32_t idS = idesc_bf16_f32(128, KT, false);
-        constexpr uint32_t idO = idesc_bf16_f32(128, D, true);
+        constexpr uint32_t idS = idesc_f16kind_f32(128, KT, false, !C::FP8);
+        constexpr uint32_t idO = idesc_f16kind_f32(128, D, true, !C::FP8);
         auto issue_s = [&](int t, int jj) {
             if (lane == 0) {
                 tc_fence_after();
@@ -284,7 +442,8 @@ __global__ void __launch_bounds__(C::NT, 1)
             const int s = j % NS, jn = j + 1, sn = jn % NS;
             if (!wait(&vfull[s], (j / NS) & 1)) break;
             const int kv0 = (jt0 + j) * KT;
-            if (kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
+            if (!C::FP8 && kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
+                // (the converters of an E4M3 cache write those rows as zeros)
                 uint8_t *vt = sV + s * C::KTILE;
                 for (int r = max(L - kv0, 0) + lane; r < KT; r += 32)
 #pragma unroll
@@ -346,7 +505,9 @@ __global__ void __launch_bounds__(C::NT, 1)
         const int ip = i0 + t * C::QPOS + r / G;
         const bool row_valid = ip < clen;
         const int pos = shared ? pfx - 1 : pfx + ip;  // last key the row attends
-        const float sl2 = a.scale * kLog2e * (a.k_scale ? a.k_scale[kvh] : 1.f);
+        // log2 units; an E4M3 row also undoes its query scale 2^qexp
+        const float sl2 = a.scale * kLog2e * (a.k_scale ? a.k_scale[kvh] : 1.f) *
+                          __uint_as_float((uint32_t)(127 - qexp) << 23);
         const uint32_t lane_base = tmem + ((uint32_t)((w & 3) * 32) << 16);
         const uint32_t scol = t * KT + half * SCOL;            // this thread's S columns
         const uint32_t pcol = t * KT + half * (SCOL / 2);      // its P words (two bf16 each)
@@ -413,12 +574,20 @@ __global__ void __launch_bounds__(C::NT, 1)
                 for (int e = 0; e < 64; e += 2) {
                     const float2 x = ffma2(make_float2(sv[64 * h + e], sv[64 * h + e + 1]), sc2, nb2);
                     const float2 pp = ((e / 2) % 8 < kEmuPairs) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
-                    const __nv_bfloat162 bb = __floats2bfloat162_rn(pp.x, pp.y);
-                    const uint32_t wb = *reinterpret_cast<const uint32_t *>(&bb);
-                    pk[e / 2] = wb;
-                    // the normaliser sums the probabilities as rounded for P.V,
-                    // so the output is an exact weighted mean of V rows
-                    sum2 = fadd2(sum2, make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
+                    if constexpr (!C::FP8) {
+                        const __nv_bfloat162 bb = __floats2bfloat162_rn(pp.x, pp.y);
+                        const uint32_t wb = *reinterpret_cast<const uint32_t *>(&bb);
+                        pk[e / 2] = wb;
+                        // the normaliser sums the probabilities as rounded for
+                        // P.V, so the output is an exact weighted mean of V rows
+                        sum2 = fadd2(sum2, make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
+                    } else {
+                        // f16 P (11 significant bits); the normaliser sums the
+                        // unrounded values (at most 2^-11 relative apart)
+                        const __half2 hh = __floats2half2_rn(pp.x, pp.y);
+                        pk[e / 2] = *reinterpret_cast<const uint32_t *>(&hh);
+                        sum2 = fadd2(sum2, pp);
+                    }
                 }
                 tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
             }
@@ -453,9 +622,9 @@ __global__ void __launch_bounds__(C::NT, 1)
                 const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
                 __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;
                 const float inv = (l > 0.f) ? 1.f / l : 0.f;
+                const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;  // E4M3 V scale (1 for bf16)
                 if (shared) {
                     // split-K piece kz of the row: normalised fp32 output and log2-sum-exp
-                    const float vs = a.v_scale ? a.v_scale[kvh] : 1.f;
                     float *wo = a.ws_o + (grow * a.max_parts + kz) * D + half * OCOL;
 #pragma unroll
                     for (int q = 0; q < OCOL / 32; ++q) {
@@ -484,7 +653,7 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
                                 for (int u = 0; u < 4; ++u) {
                                     const __nv_bfloat162 bb =
-                                        __floats2bfloat162_rn(o[e + 2 * u] * inv, o[e + 2 * u + 1] * inv);
+                                        __floats2bfloat162_rn(o[e + 2 * u] * inv * vs, o[e + 2 * u + 1] * inv * vs);
                                     wds[u] = *reinterpret_cast<const uint32_t *>(&bb);
                                 }
                                 *reinterpret_cast<uint4 *>(dst + 32 * q + e) =
@@ -533,6 +702,21 @@ bool cache_map(CUtensorMap *map, const void *base, int64_t rows, int D) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An E4M3 cache seen as a 2-D byte tensor [num_blocks*Hkv*16 rows][D]; a box
+// is 16 rows (one block of one kv head) x D bytes, unswizzled (rows land
+// row-major in the staging area).
+bool code_map(CUtensorMap *map, const void *base, int64_t rows, int D) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D};
+    const cuuint32_t box[2] = {(cuuint32_t)D, 16};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class C>
 cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
     static std::mutex mu;
@@ -551,19 +735,20 @@ cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
     }
     CUtensorMap tk, tv;
     const int64_t rows = a.num_blocks * a.Hkv * 16;
-    if (!cache_map(&tk, a.k_cache, rows, C::D) || !cache_map(&tv, a.v_cache, rows, C::D)) return cudaErrorInvalidValue;
+    auto map = C::FP8 ? code_map : cache_map;
+    if (!map(&tk, a.k_cache, rows, C::D) || !map(&tv, a.v_cache, rows, C::D)) return cudaErrorInvalidValue;
     dim3 grid((a.max_q_len + C::NQ * C::QPOS - 1) / (C::NQ * C::QPOS), a.Hkv,
               a.shared_len > 0 ? std::max(a.key_splits, 1) : a.n_chunks);
     return launch_pdl(prefill_kernel<C>, grid, dim3(C::NT), C::SMEM, st, a, tk, tv);
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t prefill_by_group(const PrefillArgs &a, cudaStream_t st) {
     switch (a.Hq / a.Hkv) {
-        case 1: return run_prefill<PCfg<D, 1>>(a, st);
-        case 2: return run_prefill<PCfg<D, 2>>(a, st);
-        case 4: return run_prefill<PCfg<D, 4>>(a, st);
-        case 8: return run_prefill<PCfg<D, 8>>(a, st);
+        case 1: return run_prefill<PCfg<D, 1, FP8>>(a, st);
+        case 2: return run_prefill<PCfg<D, 2, FP8>>(a, st);
+        case 4: return run_prefill<PCfg<D, 4, FP8>>(a, st);
+        case 8: return run_prefill<PCfg<D, 8, FP8>>(a, st);
         default: return cudaErrorNotSupported;
     }
 }
@@ -571,8 +756,9 @@ cudaError_t prefill_by_group(const PrefillArgs &a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t st) {
-    if (a.D == 128) return prefill_by_group<128>(a, st);
-    if (a.D == 64) return prefill_by_group<64>(a, st);
+    if (a.fp8 && (!a.k_scale || !a.v_scale)) return cudaErrorInvalidValue;
+    if (a.D == 128) return a.fp8 ? prefill_by_group<128, true>(a, st) : prefill_by_group<128, false>(a, st);
+    if (a.D == 64) return a.fp8 ? prefill_by_group<64, true>(a, st) : prefill_by_group<64, false>(a, st);
     return cudaErrorNotSupported;
 }
 

@@ -29,12 +29,13 @@ PA_DEVICE uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t 
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 inputs and fp32 accumulate.
-// b_mn_major: B operand stored with N contiguous (else K contiguous).
-constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// Instruction descriptor for kind::f16 with fp32 accumulate; A and B both
+// bf16 (bf16 = true) or both f16.  b_mn_major: B operand stored with N
+// contiguous (else K contiguous).
+constexpr uint32_t idesc_f16kind_f32(int M, int N, bool b_mn_major, bool bf16) {
     return (1u << 4)                      // D format: f32
-           | (1u << 7)                    // A format: bf16
-           | (1u << 10)                   // B format: bf16
+           | ((bf16 ? 1u : 0u) << 7)      // A format: bf16 (1) or f16 (0)
+           | ((bf16 ? 1u : 0u) << 10)     // B format: the same type as A
            | ((b_mn_major ? 1u : 0u) << 16)
            | ((uint32_t)(N >> 3) << 17)
            | ((uint32_t)(M >> 4) << 24);

@@ -129,12 +129,16 @@ class StepExecutor:
         self.ws = None
 
     def workspace_bytes(self, plan: StepPlan) -> int:
+        """Workspace a step needs: for plain decode of its tables, and for the
+        cascade where it takes one (the larger of the two, so that the same
+        step can also run through plain decode)."""
         maxb = plan.decode_tables.shape[1]
         B = max(plan.num_decode, 1)
+        n = ops.decode_workspace_size(B, self.Hq, self.D, maxb, self.partition)
         pb = cascade_blocks(plan, self.cascade)
         if pb:
-            return ops.cascade_workspace_size(B, self.Hq, maxb, pb, self.k_cache)
-        return ops.decode_workspace_size(B, self.Hq, self.D, maxb, self.partition)
+            n = max(n, ops.cascade_workspace_size(B, self.Hq, maxb, pb, self.k_cache))
+        return n
 
     def reserve(self, plans):
         import torch

@@ -244,10 +244,11 @@ class PrefillCase:
 
 
 def make_prefill_case(seed, chunk_lens, prefix_lens, Hq, Hkv, D, num_blocks=None, pool_factor=1.1,
-                      name="prefill"):
+                      name="prefill", fp8=False):
     """Chunks with the given lengths over existing prefixes.  The prefix
-    tokens are already in the cache (random N(0,1) contents); the chunks' own
-    K/V come as new tokens with their slot mapping (write them first)."""
+    tokens are already in the cache (random N(0,1) contents; with ``fp8`` as
+    E4M3 codes with per-head scales amax/448); the chunks' own K/V come as
+    new bf16 tokens with their slot mapping (write them first)."""
     rng = np.random.default_rng(seed)
     cl = np.asarray(chunk_lens, np.int32)
     pl = np.asarray(prefix_lens, np.int32)
@@ -261,15 +262,20 @@ def make_prefill_case(seed, chunk_lens, prefix_lens, Hq, Hkv, D, num_blocks=None
     total = int(cu[-1])
     q = normal_bf16(rng, (total, Hq, D))
     shape = (nb, Hkv, BLOCK_SIZE, D)
-    kc = normal_bf16(rng, shape)
-    vc = normal_bf16(rng, shape)
+    ks = vs = None
+    if fp8:
+        kc, ks = fp8_cache_from_normal(rng, shape)
+        vc, vs = fp8_cache_from_normal(rng, shape)
+    else:
+        kc = normal_bf16(rng, shape)
+        vc = normal_bf16(rng, shape)
     nk = normal_bf16(rng, (total, Hkv, D))
     nv = normal_bf16(rng, (total, Hkv, D))
     pos = np.concatenate([np.arange(pl[c], pl[c] + cl[c], dtype=np.int64) for c in range(len(cl))]) \
         if total else np.zeros(0, np.int64)
     rows = np.repeat(np.arange(len(cl)), cl)
     slots = bt[rows, pos // BLOCK_SIZE].astype(np.int64) * BLOCK_SIZE + pos % BLOCK_SIZE
-    return PrefillCase(name, q, cu, pl, bt, kc, vc, 1.0 / math.sqrt(D), nk, nv, slots)
+    return PrefillCase(name, q, cu, pl, bt, kc, vc, 1.0 / math.sqrt(D), nk, nv, slots, ks, vs)
 
 
 def mixed_step(seed=0, n_decode=192, n_chunks=8, chunk=512):

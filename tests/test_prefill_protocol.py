@@ -31,12 +31,23 @@ class Barrier:
             self.pending = self.count
 
 
-def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False):
-    """Run random schedules; return None or a description of the first violation."""
+def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False, fp8=False, early_refill=False):
+    """Run random schedules; return None or a description of the first violation.
+
+    fp8: the loader of an E4M3 cache -- one warp issues the TMA of each
+    tile's codes into the slot's staging area ("kload"/"vload" complete when
+    they land), both loader warps widen them into the slot and arrive on
+    full (count 2 here, one per warp); the slot of tile j-1 is refilled with
+    tile j-1+nslot once its empty barrier completes.  early_refill (a planted
+    mistake): refill the slot of tile j with tile j+nslot before its MMAs
+    are done."""
     nq, ntiles = len(ntl), max(ntl)
     for seed in range(seeds):
         rnd = random.Random(seed)
-        ring = {k: [Barrier(f"{k}{i}") for i in range(nslot)] for k in ("kfull", "kempty", "vfull", "vempty")}
+        ring = {k: [Barrier(f"{k}{i}", 2 if fp8 and k in ("kfull", "vfull") else 1) for i in range(nslot)]
+                for k in ("kfull", "kempty", "vfull", "vempty", "kload", "vload")}
+        consumed = {"k": [-1] * nslot, "v": [-1] * nslot}  # last tile whose MMAs read the slot, per slot
+        loaded = {"k": [-1] * nslot, "v": [-1] * nslot}    # tile whose codes sit in the slot
         tile = {k: [Barrier(f"{k}{t}") for t in range(nq)] for k in ("sfull", "pfull", "odone", "ofinal")}
         pending = []       # asynchronous completions, delivered in issue order
         pv_done = [-1] * nq  # last tile j whose P.V has completed, per query tile
@@ -57,6 +68,55 @@ def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False):
                         yield ring[kind + "empty"][s], use - 1
                     pending.append(ring[kind + "full"][s])
 
+        class Landed:  # the TMA of tile j's codes lands in slot s
+            def __init__(self, kind, s, j):
+                self.kind, self.s, self.j = kind, s, j
+
+            def arrive(self):
+                loaded[self.kind][self.s] = self.j
+                ring[self.kind + "load"][self.s].arrive()
+
+        def issue(kind, j):
+            s = j % nslot
+            if j >= nslot and consumed[kind][s] < j - nslot:
+                violation.append(f"{kind} codes of tile {j} issued over tile {j - nslot} still in use")
+            pending.append(Landed(kind, s, j))
+
+        violation = []
+
+        def fp8_issuer():
+            for j in range(min(nslot, ntiles)):
+                issue("k", j)
+                issue("v", j)
+            for j in range(ntiles):
+                for kind in ("k", "v"):
+                    yield ring[kind + "load"][j % nslot], j // nslot
+                    if loaded[kind][j % nslot] != j:
+                        yield None, f"{kind} tile {j} widened from the codes of tile {loaded[kind][j % nslot]}"
+                    ring[kind + "full"][j % nslot].arrive()
+                jr, jd = (j + nslot, j) if early_refill else (j - 1 + nslot, j - 1)
+                if jd >= 0 and jr < ntiles:
+                    for kind in ("k", "v"):
+                        if not early_refill:
+                            yield ring[kind + "empty"][jd % nslot], jd // nslot
+                        issue(kind, jr)
+                if violation:
+                    yield None, violation[0]
+
+        def fp8_widener():  # the second loader warp: widens the same tiles
+            for j in range(ntiles):
+                for kind in ("k", "v"):
+                    yield ring[kind + "load"][j % nslot], j // nslot
+                    ring[kind + "full"][j % nslot].arrive()
+
+        class Consumed:  # the MMAs reading a slot's tile have completed
+            def __init__(self, kind, s, j, bar):
+                self.kind, self.s, self.j, self.bar = kind, s, j, bar
+
+            def arrive(self):
+                consumed[self.kind][self.s] = max(consumed[self.kind][self.s], self.j)
+                self.bar.arrive()
+
         def mma():
             violation = []
             if ntiles:
@@ -64,7 +124,7 @@ def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False):
                 for t in range(nq):
                     if ntl[t]:
                         pending.append(tile["sfull"][t])
-                pending.append(ring["kempty"][0])
+                pending.append(Consumed("k", 0, 0, ring["kempty"][0]))
             for j in range(ntiles):
                 s, jn = j % nslot, j + 1
                 yield ring["vfull"][s], j // nslot
@@ -85,11 +145,11 @@ def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False):
                             violation.append(f"S_{t}({jn}) issued before P_{t}({j}).V completed")
                             yield None, violation[-1]
                         pending.append(tile["sfull"][t])
-                pending.append(ring["vempty"][s])
+                pending.append(Consumed("v", s, j, ring["vempty"][s]))
                 if jn < ntiles:
                     if not kready:
                         yield ring["kfull"][jn % nslot], jn // nslot
-                    pending.append(ring["kempty"][jn % nslot])
+                    pending.append(Consumed("k", jn % nslot, jn, ring["kempty"][jn % nslot]))
 
         def softmax(t):
             for j in range(ntl[t]):
@@ -98,7 +158,8 @@ def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False):
             if ntl[t]:
                 yield tile["ofinal"][t], 0
 
-        actors = {"load": loader(), "mma": mma(), **{f"softmax{t}": softmax(t) for t in range(nq)}}
+        loaders = {"issue": fp8_issuer(), "widen": fp8_widener()} if fp8 else {"load": loader()}
+        actors = {**loaders, "mma": mma(), **{f"softmax{t}": softmax(t) for t in range(nq)}}
         waiting = {k: None for k in actors}
         done = set()
         while len(done) < len(actors):
@@ -143,6 +204,22 @@ SHAPES = [(1, 0), (3, 0), (2, 3), (5, 6), (9, 10), (1, 1), (4, 4), (8, 8)]
 @pytest.mark.parametrize("nslot", [2, 4])
 def test_protocol_has_no_deadlock_aliasing_or_overwrite(ntl, nslot):
     assert explore(list(ntl), nslot, seeds=120) is None
+
+
+@pytest.mark.parametrize("ntl", SHAPES)
+@pytest.mark.parametrize("nslot", [2])
+def test_fp8_loader_protocol(ntl, nslot):
+    """The E4M3 loader (TMA of codes into staging, widening by two warps,
+    refill of a slot once its previous tile's MMAs are done): no deadlock, no
+    stale phase, no tile widened from another tile's codes, no codes issued
+    over a tile still being read."""
+    assert explore(list(ntl), nslot, seeds=120, fp8=True) is None
+
+
+def test_fp8_refill_before_the_slot_is_free_is_caught():
+    found = [explore([6, 7], 2, seeds=200, fp8=True, early_refill=True),
+             explore([9, 10], 2, seeds=200, fp8=True, early_refill=True)]
+    assert any(found), "refilling a slot before its MMAs completed went unnoticed"
 
 
 def test_a_skipped_o_done_wait_is_caught():
