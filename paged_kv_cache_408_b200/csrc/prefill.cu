@@ -582,11 +582,16 @@ __global__ void __launch_bounds__(C::NT, 1)
                         // P.V, so the output is an exact weighted mean of V rows
                         sum2 = fadd2(sum2, make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
                     } else {
-                        // f16 P (11 significant bits); the normaliser sums the
-                        // unrounded values (at most 2^-11 relative apart)
+                        // f16 P; the normaliser sums it as rounded too.  An f16
+                        // moved up 13 bits is an fp32 of the same significand
+                        // and 2^-112 times the value (f16 subnormals and zero
+                        // included), so the sum is kept scaled by 2^-112 and
+                        // scaled back once, in the epilogue
                         const __half2 hh = __floats2half2_rn(pp.x, pp.y);
-                        pk[e / 2] = *reinterpret_cast<const uint32_t *>(&hh);
-                        sum2 = fadd2(sum2, pp);
+                        const uint32_t wh = *reinterpret_cast<const uint32_t *>(&hh);
+                        pk[e / 2] = wh;
+                        sum2 = fadd2(sum2, make_float2(__uint_as_float((wh & 0xffffu) << 13),
+                                                       __uint_as_float((wh >> 16) << 13)));
                     }
                 }
                 tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
@@ -617,6 +622,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             l = 0.f;
 #pragma unroll
             for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
+            if constexpr (C::FP8) l *= 0x1p112f;  // the f16 sum was kept scaled by 2^-112
             if (wait(&ofinal[t], 0)) {
                 tc_fence_after();
                 const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
