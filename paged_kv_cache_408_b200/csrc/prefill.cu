@@ -137,8 +137,20 @@ __global__ void __launch_bounds__(C::NT, 1)
     float *xch = reinterpret_cast<float *>(smem + C::OFF_X);  // [3][NQ][NSPLIT][128]: max (2 parities), sum
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int c = a.shared_len > 0 ? 0 : blockIdx.z, kvh = blockIdx.y;
-    const int i0 = blockIdx.x * (NQ * C::QPOS);
+    // CTA -> (chunk c, kv head, query tiles from i0).  CTAs start in the order
+    // of their linear index (x fastest); in a causal chunk a later query tile
+    // attends more keys, so each chunk's CTAs are taken longest first
+    // (query-tile pair descending, kv heads within), which leaves shorter
+    // work for the end of the grid.  Shared-prefix mode keeps the grid as is.
+    int c = 0, kvh = blockIdx.y, qx = blockIdx.x;
+    if (a.shared_len <= 0) {
+        const int nx = gridDim.x, lin = blockIdx.x + nx * (blockIdx.y + gridDim.y * blockIdx.z);
+        const int rem = lin % (nx * gridDim.y);
+        c = lin / (nx * gridDim.y);
+        qx = nx - 1 - rem / gridDim.y;
+        kvh = rem % gridDim.y;
+    }
+    const int i0 = qx * (NQ * C::QPOS);
     pdl_trigger();
     pdl_wait();
     const uint64_t deadline = wait_deadline();  // shared by every wait of this launch

@@ -314,3 +314,34 @@ def test_kv_accounting_shows_paging_waste_and_sharing():
     assert acc["sequences"] == 256 and acc["tokens_per_block_capacity"] > 5
     import json
     json.dumps(acc)  # bench.py prints it in its JSON line
+
+
+def test_mixed_trace_plans_carry_prefill_chunks():
+    """The mixed trace drives chunked prefill through the scheduler: step 0 is
+    192 decode rows plus 8 chunks of 512 tokens over cached prefixes in
+    [0, 4096]; every later step keeps 8 prompts in prefill, each advancing by
+    a chunk of at most 512 tokens within the 8192-token budget, decode rows
+    first; the invariants of the pool hold after every step."""
+    from paged_kv_cache_408_b200 import traces
+    tr = traces.mixed(0)
+    plans = []
+    for _ in range(12):
+        plans += tr.plans(1)
+        R.check_invariants(tr.sched)
+    p0 = plans[0]
+    assert p0.num_decode == 192 and len(p0.prefill_ids) == 8 and p0.num_prefill_tokens == 8 * 512
+    assert (np.diff(p0.prefill_cu) == 512).all()
+    assert ((p0.prefill_prefix >= 0) & (p0.prefill_prefix <= 4096)).all()
+    for p in plans:
+        chunks = np.diff(p.prefill_cu)
+        assert len(chunks) == 8 and (chunks > 0).all() and (chunks <= 512).all()
+        assert p.num_decode + p.num_prefill_tokens <= 8192
+        # slots: decode tokens first (one per row), then each chunk's tokens in order
+        assert len(p.slots) == p.num_decode + p.num_prefill_tokens
+        # a chunk's tables cover its prefix and the chunk itself
+        for c in range(len(chunks)):
+            need = (int(p.prefill_prefix[c]) + int(chunks[c]) + 15) // 16
+            assert (p.prefill_tables[c, :need] >= 0).all()
+    # prompts finish and join the decode batch; new prompts start from an empty prefix
+    assert max(p.num_decode for p in plans) > 192
+    assert any((p.prefill_prefix == 0).any() for p in plans[1:])
