@@ -29,16 +29,11 @@
 //    tensor core's shared-memory reads are only Q, K and V.  The two query
 //    tiles alternate: the tensor core works on one tile's products while
 //    the other tile's softmax runs.
-//  * S_t(j+1) is issued in two halves of 64 keys: the upper half writes S
-//    columns P_t never occupies and follows O_t += P_t(j) V_j at once; the
-//    lower half overwrites P_t and is issued only after that P.V has
-//    completed -- the upper half keeps the tensor core busy meanwhile, so
-//    the pipe does not drain at that wait (a drained tcgen05 pipe takes
-//    several hundred clocks to refill).  When softmax t sees S_t(j+1) the
-//    previous P.V is therefore done and a rescale of its O row in TMEM is
-//    safe.  The MMA warp issues, per tile in turn, P.V as soon as P arrives
-//    and then the tile's next S, so a tile never waits for the other tile's
-//    softmax.
+//  * S_t(j+1) is issued only after O_t += P_t(j) V_j has completed (it
+//    overwrites P_t), so when softmax t sees S_t(j+1) the previous P.V is
+//    done and a rescale of its O row in TMEM is safe.  The MMA warp issues,
+//    per tile in turn, P.V as soon as P arrives and then the tile's next S,
+//    so a tile never waits for the other tile's softmax.
 //  * Softmax applies the causal mask only on tiles that reach past the
 //    row's position, moves the running max only when it grows by more than
 //    8 (log2 units), and computes P with one packed FMA and one
@@ -70,7 +65,7 @@ constexpr float kRescaleThreshold = 8.0f;
 // through the FMA-pipe exponential (fastexp.cuh) and the rest through MUFU:
 // with head_dim 128 MUFU alone needs as many clocks per tile as the two
 // MMAs of a query tile, which would leave the tensor core waiting.
-constexpr int kEmuPairs = 0;
+constexpr int kEmuPairs = 3;
 
 template <int D_, int G_, bool FP8_>
 struct PCfg {
@@ -434,35 +429,24 @@ __global__ void __launch_bounds__(C::NT, 1)
         // as soon as that P.V has completed (S_t(j+1) overwrites P_t).  Tile
         // 0's next scores never wait for tile 1's softmax, and tile 1 stays
         // half a step behind tile 0, so the two softmaxes use MUFU in turns.
-        constexpr uint32_t idS = idesc_f16kind_f32(128, KT / 2, false, !C::FP8);
+        constexpr uint32_t idS = idesc_f16kind_f32(128, KT, false, !C::FP8);
         constexpr uint32_t idO = idesc_f16kind_f32(128, D, true, !C::FP8);
-        // S_t = Q_t K^T in two halves of KT/2 keys (N = KT/2 MMAs): part 1
-        // writes S columns [KT/2, KT), which P_t (packed into the first KT/2
-        // columns) never occupies, so it is issued right behind O_t += P_t V
-        // without waiting; part 0 overwrites P_t and waits for that P.V to
-        // complete -- while part 1 keeps the tensor core busy, so the pipe
-        // never drains at that wait.  S full is committed after part 0.
-        auto issue_s = [&](int t, int jj, int part) {
+        auto issue_s = [&](int t, int jj) {
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t q0 = smem_addr(sQ + t * C::QTILE);
-                const uint32_t k0 = smem_addr(sK + (jj % NS) * C::KTILE) + part * (KT / 2) * 128;
+                const uint32_t q0 = smem_addr(sQ + t * C::QTILE), k0 = smem_addr(sK + (jj % NS) * C::KTILE);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc_mma_bf16(tmem + t * KT + part * (KT / 2),
-                                smem_desc_sw128(q0 + (kk / 4) * C::QATOM + (kk % 4) * 32, 16, 1024),
+                    tc_mma_bf16(tmem + t * KT, smem_desc_sw128(q0 + (kk / 4) * C::QATOM + (kk % 4) * 32, 16, 1024),
                                 smem_desc_sw128(k0 + (kk / 4) * C::KATOM + (kk % 4) * 32, 16, 1024), idS, kk > 0);
-                if (part == 0) tc_commit(&sfull[t]);
+                tc_commit(&sfull[t]);
             }
             __syncwarp();
         };
         if (ntiles > 0 && wait(&kfull[0], 0)) {
 #pragma unroll
             for (int t = 0; t < NQ; ++t)
-                if (ntl[t] > 0) {
-                    issue_s(t, 0, 1);
-                    issue_s(t, 0, 0);
-                }
+                if (ntl[t] > 0) issue_s(t, 0);
             if (lane == 0) tc_commit(&kempty[0]);
             __syncwarp();
         }
@@ -505,9 +489,8 @@ __global__ void __launch_bounds__(C::NT, 1)
                         if (!wait(&kfull[sn], (jn / NS) & 1)) break;
                         kready = true;
                     }
-                    issue_s(t, jn, 1);                   // columns P_t(j) does not use
-                    if (!wait(&odone[t], j & 1)) break;  // P_t(j) consumed by its P.V
-                    issue_s(t, jn, 0);
+                    if (!wait(&odone[t], j & 1)) break;  // P_t(j) consumed
+                    issue_s(t, jn);
                 }
             }
             if (!ok) break;
@@ -570,13 +553,9 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
                 for (int e = 0; e < SCOL; ++e) sv[e] = (row_valid && kv0 + e <= pos) ? sv[e] : -INFINITY;
             }
-            // the thread's max as four independent chains (a short dependency chain)
-            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float mraw = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < SCOL; e += 8)
-#pragma unroll
-                for (int u = 0; u < 4; ++u) mq[u] = fmax3(mq[u], sv[e + 2 * u], sv[e + 2 * u + 1]);
-            float mraw = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            for (int e = 0; e < SCOL; e += 2) mraw = fmax3(mraw, sv[e], sv[e + 1]);
             // the row's max over its threads; after this barrier every thread
             // of the row has read its S columns, so P may overwrite them
             *xslot(j & 1, half) = mraw;
@@ -599,7 +578,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             // score; masked scores are -inf and give 2^-inf = 0
             const float mb = (m == -INFINITY) ? 0.f : m;
             const float2 sc2 = make_float2(sl2, sl2), nb2 = make_float2(-mb, -mb);
-            float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // two chains
+            float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < SCOL / 64; ++h) {
                 uint32_t pk[32];
@@ -613,8 +592,7 @@ __global__ void __launch_bounds__(C::NT, 1)
                         pk[e / 2] = wb;
                         // the normaliser sums the probabilities as rounded for
                         // P.V, so the output is an exact weighted mean of V rows
-                        sum2[(e / 2) & 1] = fadd2(sum2[(e / 2) & 1],
-                                                  make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
+                        sum2 = fadd2(sum2, make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
                     } else {
                         // f16 P; the normaliser sums it as rounded too.  An f16
                         // moved up 13 bits is an fp32 of the same significand
@@ -624,13 +602,13 @@ __global__ void __launch_bounds__(C::NT, 1)
                         const __half2 hh = __floats2half2_rn(pp.x, pp.y);
                         const uint32_t wh = *reinterpret_cast<const uint32_t *>(&hh);
                         pk[e / 2] = wh;
-                        sum2[(e / 2) & 1] = fadd2(sum2[(e / 2) & 1], make_float2(__uint_as_float((wh & 0xffffu) << 13),
-                                                                                 __uint_as_float((wh >> 16) << 13)));
+                        sum2 = fadd2(sum2, make_float2(__uint_as_float((wh & 0xffffu) << 13),
+                                                       __uint_as_float((wh >> 16) << 13)));
                     }
                 }
                 tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
             }
-            l += (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);  // this thread's keys; rows combine at the end
+            l += sum2.x + sum2.y;  // this thread's keys; the row sum is combined at the end
             // O_t holds P.V up to tile j-1, complete (S_t(j) was issued after it):
             // rescale in TMEM; tcgen05.ld/st are warp-collective, so the warp
             // rescales if any of its rows needs it

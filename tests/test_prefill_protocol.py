@@ -5,10 +5,8 @@ GPU here).
 Actors, as in `prefill_kernel` (csrc/prefill.cu): the TMA warp fills K and V
 ring slots (waiting on the slot's "empty" barrier before a refill); the MMA
 warp issues, per key tile j, P_t(j).V_j for each query tile t as soon as that
-tile's softmax has written P_t(j), then the upper half of S_t(j+1) =
-Q_t.K_{j+1}^T (columns P_t does not occupy; no barrier involved, so the model
-has no step for it), then the lower half once that P.V has completed (it
-overwrites P_t(j) in TMEM), then commits S full; one softmax actor per
+tile's softmax has written P_t(j), then S_t(j+1) = Q_t.K_{j+1}^T once that
+P.V has completed (S_t(j+1) overwrites P_t(j) in TMEM); one softmax actor per
 query tile waits for S_t(j), writes P_t(j) and signals it.  MMA completions
 (tcgen05.commit) and copy completions arrive later, in issue order.
 
