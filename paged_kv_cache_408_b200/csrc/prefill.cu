@@ -65,7 +65,7 @@ constexpr float kRescaleThreshold = 8.0f;
 // through the FMA-pipe exponential (fastexp.cuh) and the rest through MUFU:
 // with head_dim 128 MUFU alone needs as many clocks per tile as the two
 // MMAs of a query tile, which would leave the tensor core waiting.
-constexpr int kEmuPairs = 3;
+constexpr int kEmuPairs = 0;
 
 template <int D_, int G_, bool FP8_>
 struct PCfg {
