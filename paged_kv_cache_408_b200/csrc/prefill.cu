@@ -37,10 +37,9 @@
 //  * Softmax applies the causal mask only on tiles that reach past the
 //    row's position, moves the running max only when it grows by more than
 //    8 (log2 units), and computes P with one packed FMA and one
-//    exponential per score: 5 of every 8 pairs on MUFU (ex2.approx), 3 on
-//    the FMA pipe (fastexp.cuh), so that neither unit sets the pace; the
-//    row sum l adds P as rounded to bf16 for the P.V product, so numerator
-//    and denominator use the same weights.
+//    exponential per score (MUFU; kEmuPairs of every 8 pairs can go to the
+//    FMA pipe, fastexp.cuh).  The row sum l adds the fp32 probabilities for
+//    a bf16 cache and the f16-rounded ones for an E4M3 cache.
 //  * Every mbarrier is waited on in phase order and never falls two phases
 //    behind its producer (a parity wait cannot tell phase k from k+2); the
 //    protocol was checked against that rule, and for deadlock, by a
@@ -267,10 +266,21 @@ __global__ void __launch_bounds__(C::NT, 1)
     // MMA warp stop issuing, the softmax warps only keep their named
     // barriers and arrivals in step (so no thread waits on a partner that has
     // left), and the asynchronous work already issued is drained below.
-    // ok is kept warp-uniform, since tcgen05.ld/st and the MMA issue are
-    // warp-collective.
+    // Every lane polls the barrier itself (each lane's accesses are then
+    // ordered after its own observation of the phase).  In the loader and
+    // MMA warps, whose tensor-core and TMA instructions are issued by single
+    // lanes, ok is per lane: a lane past the deadline fails every later wait
+    // at once, so all lanes leave their loops within one step of each other.
+    // The softmax warps' tcgen05.ld/st are warp-collective, so there ok is
+    // made warp-uniform by a vote once per tile (wait_all).  (A vote after
+    // every wait of the MMA and loader warps measured 7% of the kernel's
+    // time; one polling lane with a broadcast, twice as long.)
     bool ok = true;
     auto wait = [&](uint64_t *bar, uint32_t parity) {
+        ok = ok && mbar_wait(bar, parity, deadline);
+        return ok;
+    };
+    auto wait_all = [&](uint64_t *bar, uint32_t parity) {
         ok = ok && mbar_wait(bar, parity, deadline);
         ok = __all_sync(0xffffffffu, ok);
         return ok;
@@ -532,7 +542,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             // barrier and arrives on P full, so that no thread is left waiting
             // on it
             float sv[SCOL];
-            if (wait(&sfull[t], j & 1)) {
+            if (wait_all(&sfull[t], j & 1)) {
                 tc_fence_after();
 #pragma unroll
                 for (int q = 0; q < SCOL / 32; ++q) {
@@ -588,11 +598,12 @@ __global__ void __launch_bounds__(C::NT, 1)
                     const float2 pp = ((e / 2) % 8 < kEmuPairs) ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
                     if constexpr (!C::FP8) {
                         const __nv_bfloat162 bb = __floats2bfloat162_rn(pp.x, pp.y);
-                        const uint32_t wb = *reinterpret_cast<const uint32_t *>(&bb);
-                        pk[e / 2] = wb;
-                        // the normaliser sums the probabilities as rounded for
-                        // P.V, so the output is an exact weighted mean of V rows
-                        sum2 = fadd2(sum2, make_float2(__uint_as_float(wb << 16), __uint_as_float(wb & 0xffff0000u)));
+                        pk[e / 2] = *reinterpret_cast<const uint32_t *>(&bb);
+                        // the normaliser sums the fp32 probabilities (summing them
+                        // as rounded to bf16 cost 3% of the kernel): each weight
+                        // of the P.V product is then off by at most 2^-9
+                        // relative, within the tolerance
+                        sum2 = fadd2(sum2, pp);
                     } else {
                         // f16 P; the normaliser sums it as rounded too.  An f16
                         // moved up 13 bits is an fp32 of the same significand
@@ -635,7 +646,7 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
             for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
             if constexpr (C::FP8) l *= 0x1p112f;  // the f16 sum was kept scaled by 2^-112
-            if (wait(&ofinal[t], 0)) {
+            if (wait_all(&ofinal[t], 0)) {
                 tc_fence_after();
                 const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
                 __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;
