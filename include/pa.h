@@ -261,9 +261,15 @@ int pa_decode_cascade(void *out, const void *q, const void *k_cache, const void 
  *   max_q_len     host upper bound on any chunk's length (sizes the grid).
  *   total_q_tokens  rows of q and out (= cu_q_lens[num_chunks]); chunks
  *                 reaching past it are rejected on the device.
+ *   k_scale, v_scale  fp32 [num_kv_heads] for an fp8 cache (required;
+ *                 PA_ERR_INVALID_ARG without them), ignored for bf16.
  * The chunk's own K/V must already be in the cache (pa_write_kv first).
- * bf16 cache only; an fp8 cache returns PA_ERR_UNSUPPORTED.  head_dim 64 or
- * 128; num_q_heads / num_kv_heads in {1,2,4,8}.
+ * bf16 cache: bf16 MMA operands.  fp8 E4M3 cache: each K/V tile is widened
+ * exactly to f16 in shared memory on its way to the tensor cores, a query
+ * row is scaled by a power of two into f16 range (exact for components
+ * within 2^-28 of the row's largest), P enters P.V as f16; fp32
+ * accumulation throughout.  head_dim 64 or 128; num_q_heads / num_kv_heads
+ * in {1,2,4,8}.
  */
 int pa_prefill_chunk(void *out, const void *q, const int32_t *cu_q_lens, const int32_t *prefix_lens,
                      const int32_t *block_tables, int32_t num_chunks, int32_t max_blocks_per_seq,
@@ -316,8 +322,10 @@ int pa_get_last_device_error(uint32_t *flags, pa_stream_t stream);
 /* Human-readable name of a pa_status value (static string). */
 const char *pa_status_string(int status);
 
-/* Library version as an integer (major*10000 + minor*100 + patch): 200 =
- * 0.2.0, which adds pa_decode_cascade and pa_decode_noalloc to 0.1.0. */
+/* Library version as an integer (major*10000 + minor*100 + patch): 300 =
+ * 0.3.0, which adds chunked prefill over an fp8 cache and the
+ * PA_MAX_BLOCKS_PER_SEQ bound to 0.2.0 (pa_decode_cascade,
+ * pa_decode_noalloc). */
 int pa_version(void);
 
 #ifdef __cplusplus

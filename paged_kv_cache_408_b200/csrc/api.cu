@@ -72,7 +72,7 @@ int pa::sm_count() {
 
 extern "C" {
 
-int pa_version(void) { return 200; }
+int pa_version(void) { return 300; }
 
 const char *pa_status_string(int status) {
     switch (status) {

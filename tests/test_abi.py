@@ -140,7 +140,7 @@ def test_cascade_workspace_size():
     # split-K pieces of the 32-block suffix (at most 32/16 + 2) plus the prefix piece, fp32 o and lse
     assert n >= 256 * 64 * 5 * (128 + 1) * 4
     rc, n8 = cascade_ws(256, 64, 160, 128, dt=1)
-    assert rc == 0 and n8 == n  # an fp8 prefix is widened inside the prefill kernel: no scratch copy
+    assert rc == 0 and n8 >= n + 2 * 128 * 8 * 16 * 128 * 2  # fp8: the prefix widened to bf16
     assert cascade_ws(256, 64, 160, 161)[0] == -1
     assert cascade_ws(256, 64, 160, -1)[0] == -1
     assert cascade_ws(256, 64, 160, 0)[1] >= ops.decode_workspace_size(256, 64, 128, 160)
