@@ -557,6 +557,60 @@ def cascade_blocks(plan, args):
     return cb(plan, not args.no_cascade)
 
 
+def static_prefill(args, device, fp8=False, n=30):
+    """The mixed step's prefill as a fixed workload (8 chunks of 512 tokens
+    over prefixes uniform in [0, 4096], 32/8 heads, d128; the chunks' K/V
+    written first), the prefill call timed alone n times, L2 flushed before
+    each: median device time and algorithmic FLOPs."""
+    import torch
+
+    from paged_kv_cache_408_b200 import inputs as I
+    from paged_kv_cache_408_b200 import ops
+    pc = I.mixed_step_prefill(args.seed, fp8=fp8)
+    if fp8:
+        kc, vc = torch.from_numpy(pc.k_cache).to(device), torch.from_numpy(pc.v_cache).to(device)
+        ks, vs = torch.from_numpy(pc.k_scale).to(device), torch.from_numpy(pc.v_scale).to(device)
+    else:
+        def bf(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+        kc, vc = bf(pc.k_cache), bf(pc.v_cache)
+        ks = vs = None
+
+    def bfq(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(device)
+
+    ops.write_kv(bfq(pc.new_k), bfq(pc.new_v), torch.from_numpy(pc.slot_mapping).to(device), kc, vc, ks, vs)
+    q = bfq(pc.q)
+    out = torch.empty_like(q)
+    cu, pf, bt = i32(pc.cu_q), i32(pc.prefix_lens), i32(pc.block_tables)
+    flush = L2Flush(torch, device)
+    st = torch.cuda.current_stream()
+    for _ in range(3):
+        ops.prefill_chunk(out, q, cu, pf, bt, kc, vc, pc.scale, pc.max_q_len, ks, vs)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda._sleep(hold_cycles(n))
+    for e0, e1 in ev:
+        flush()
+        e0.record(st)
+        ops.prefill_chunk(out, q, cu, pf, bt, kc, vc, pc.scale, pc.max_q_len, ks, vs)
+        e1.record(st)
+    torch.cuda.synchronize()
+    if ops.get_last_device_error():
+        raise RuntimeError("device status word set during the static prefill step")
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    fl = prefill_flops(pc.cu_q, pc.prefix_lens, 32, 128)
+    peak, kind = tensor_peak()
+    tfl = fl / (ms / 1e3) / 1e12
+    return {"workload": "8 chunks x 512 over prefixes U[0,4096] (static), 32/8 heads, d128, " +
+                        ("fp8 E4M3 cache" if fp8 else "bf16"),
+            "ms_per_launch": ms, "flops_per_launch": fl, "tflops": tfl, "frac": tfl / peak, "peak": peak,
+            "peak_kind": kind, "launches": n, "timing": "median of n calls alone, CUDA events, L2 flushed before each"}
+
+
 def prefill_block(pf):
     """The prefill call's figures: algorithmic FLOPs over its CUDA-event time,
     against the measured bf16 GEMM peak (the call is timed alone)."""
@@ -673,6 +727,9 @@ def main():
         pf = r.get("prefill") or leg
         if pf:
             line["prefill"] = prefill_block(pf)
+            if not args.no_prefill_leg:
+                line["prefill"]["static_step"] = static_prefill(args, device)
+                line["prefill"]["static_step_fp8"] = static_prefill(args, device, fp8=True)
         if world == 1 and not args.no_cpu_baseline and r.get("plans"):
             import torch as _t
             kc, vc = host_copy(r["k_cache"], _t), host_copy(r["v_cache"], _t)

@@ -294,6 +294,20 @@ def mixed_step(seed=0, n_decode=192, n_chunks=8, chunk=512):
     return dec, pre
 
 
+def mixed_step_prefill(seed=0, n_decode=192, n_chunks=8, chunk=512, fp8=False):
+    """The prefill half of ``mixed_step(seed)`` alone (the same chunk
+    prefixes), without drawing its decode half's cache; with ``fp8`` the
+    same chunks over an E4M3 cache drawn from another seed."""
+    rng = np.random.default_rng(20_000 + seed)
+    lognormal_lengths(rng, n_decode)  # the decode lengths come first in mixed_step's draw order
+    prefixes = rng.integers(0, 4097, n_chunks).astype(np.int32)
+    if fp8:
+        return make_prefill_case(seed + 543, [chunk] * n_chunks, prefixes, 32, 8, 128, fp8=True,
+                                 name="8 chunks x 512 over U[0,4096] prefixes, fp8")
+    return make_prefill_case(seed + 1, [chunk] * n_chunks, prefixes, 32, 8, 128,
+                             name="mixed: 8 chunks x 512 over U[0,4096] prefixes")
+
+
 def prefix_share(seed=0, n_seqs=256, prefix=2048, suffix_lo=16, suffix_hi=512, Hq=64, Hkv=8, D=128, fp8=True):
     """256 sequences sharing one 2048-token prefix (the same physical blocks)
     plus per-sequence suffixes uniform in [16, 512]; 64/8 heads, head_dim
