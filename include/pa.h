@@ -90,6 +90,7 @@ typedef enum pa_dtype {
 #define PA_DEVERR_BAD_LEN 0x4u    /* seq_len < 0 or > 16 * max_blocks_per_seq (cascade: < 16 * prefix_blocks) */
 #define PA_DEVERR_BAD_PAIR 0x8u   /* a copy pair outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT 0x10u   /* a bounded wait for an async copy or MMA gave up (results invalid) */
+#define PA_DEVERR_LAYOUT 0x20u    /* prefill: the CTA's shared memory did not start on a 1 KB boundary (no output written) */
 
 /* An opaque stream handle: pass a cudaStream_t. */
 typedef void *pa_stream_t;

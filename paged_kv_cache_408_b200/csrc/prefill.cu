@@ -69,7 +69,12 @@ constexpr int kEmuPairs = 0;
 template <int D_, int G_, bool FP8_>
 struct PCfg {
     static constexpr int D = D_, G = G_;
-    static constexpr bool FP8 = FP8_;             // E4M3 cache: f16 operands, K/V widened by converter warps
+    static constexpr bool FP8 = FP8_;             // E4M3 cache: f16 operands, K/V widened by the loader warps
+    // bf16 cache: P goes to shared memory and the P.V MMA reads it from
+    // there, so S_t(j+1) may be issued into S_t's TMEM columns as soon as
+    // the softmax has loaded S_t(j).  E4M3 cache: P is written over S_t's
+    // TMEM columns, and S_t(j+1) waits for P_t(j).V_j to complete.
+    static constexpr bool PSMEM = !FP8_;
     static constexpr int M = 128;                 // accumulator rows of a query tile
     static constexpr int QPOS = M / G;            // query positions per query tile
     static constexpr int NQ = 2;                  // query tiles per CTA
@@ -79,10 +84,22 @@ struct PCfg {
     static constexpr int KATOM = KT * 128;        // bytes of one atom column of a K/V tile
     static constexpr int QTILE = NATOM * QATOM;
     static constexpr int KTILE = NATOM * KATOM;
-    static constexpr int NSLOT = (D == 128 || FP8) ? 2 : 4;  // K and V ring depth
+    // K and V ring depths.  With P in shared memory and head_dim 128 the
+    // budget leaves 2 K slots and 1 V slot: K_{j+1} is requested a tile
+    // period ahead (the next scores need it early), V_j once P(j-1).V is
+    // done (P.V needs it late), so the two copies do not compete for the
+    // TMA bandwidth.  (One ring of three slots filled in read order --
+    // K_{j+1}, V_j, ... -- requests both early and measured 2.5% slower;
+    // two V slots with one P buffer shared by the query tiles, 8% slower.)
+    static constexpr int NSK = PSMEM ? (D == 128 ? 2 : 3) : 2;
+    static constexpr int NSV = PSMEM ? (D == 128 ? 1 : 3) : 2;
+    static constexpr int NPB = PSMEM ? NQ : 0;     // P buffers: one per query tile
+    static constexpr int PATOM = M * 128;         // P: one atom column = 64 keys of 128 rows
+    static constexpr int PTILE = (KT / 64) * PATOM;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + NQ * QTILE;
-    static constexpr int OFF_V = OFF_K + NSLOT * KTILE;
+    static constexpr int OFF_V = OFF_K + NSK * KTILE;
+    static constexpr int OFF_P = OFF_V + NSV * KTILE;
     static constexpr int NSPLIT = 2;              // softmax threads per accumulator row
     static constexpr int SCOL = KT / NSPLIT;      // S columns (keys) per softmax thread
     static constexpr int OCOL = D / NSPLIT;       // O columns per softmax thread
@@ -94,21 +111,35 @@ struct PCfg {
     // one atom column, so the codes get a ring of their own.
     static constexpr int STG_BYTES = KT * D;      // one tile of codes
     static constexpr bool STG_IN_PLACE = FP8 && D == 128;
-    static constexpr int OFF_STG = OFF_V + NSLOT * KTILE;
-    static constexpr int STG_RING = (FP8 && !STG_IN_PLACE) ? 2 * NSLOT * STG_BYTES : 0;
-    static constexpr int OFF_X = OFF_STG + STG_RING;  // row max / sum exchange of a row's threads
-    static constexpr int OFF_BAR = OFF_X + 3 * NQ * NSPLIT * 128 * 4;
-    // K/V full+empty; S full, P full, O done, O final; end; (E4M3) K/V codes loaded
-    static constexpr int NBAR = 4 * NSLOT + 4 * NQ + 1 + (FP8 ? 2 * NSLOT : 0);
-    static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // barriers, TMEM slot, alignment slack
+    static constexpr int OFF_STG = OFF_P + NPB * PTILE;
+    static constexpr int STG_RING = (FP8 && !STG_IN_PLACE) ? (NSK + NSV) * STG_BYTES : 0;
+    // row max exchange of a row's threads (two parities), and for an E4M3
+    // cache the row sums and query magnitudes: fp32.  With P in shared
+    // memory the maxima travel as bf16 rounded up (both threads of a row
+    // take the same rounded values, so they agree on the row's reference
+    // point) and the sums go through the query tile's buffer once O is
+    // final (every MMA that read it has completed).
+    static constexpr int OFF_X = OFF_STG + STG_RING;
+    static constexpr int X_BYTES = PSMEM ? 2 * NQ * NSPLIT * 128 * 2 : 3 * NQ * NSPLIT * 128 * 4;
+    static constexpr int OFF_BAR = OFF_X + X_BYTES;
+    // K/V full+empty; S full, P full, O done, O final; (P in shared memory)
+    // S free; end; (E4M3) K/V codes loaded
+    static constexpr int NBAR = 2 * NSK + 2 * NSV + 4 * NQ + (PSMEM ? NQ : 0) + 1 + (FP8 ? NSK + NSV : 0);
+    static constexpr int USED = OFF_BAR + NBAR * 8 + 16;  // + the TMEM address slot
+    // the tiles need a 1024-byte aligned base: slack to align it where the
+    // budget allows, else the launch requires the base aligned (it is: the
+    // dynamic shared memory of a CTA starts on a 1 KB boundary) and checks it
+    static constexpr int SLACK = USED + 1024 <= 227 * 1024 ? 1024 : 0;
+    static constexpr int SMEM = USED + SLACK;
     static constexpr int NSMW = NQ * 4 * NSPLIT;  // softmax warps
-    // loader warps: one TMA warp (bf16 cache), or four converter warps that
-    // widen E4M3 K/V rows into the operand tiles (one key row per thread)
+    // loader warps: one TMA warp (bf16 cache), or two warps that gather
+    // E4M3 K/V codes and widen them into the operand tiles
     static constexpr int NLOAD = FP8 ? 2 : 1;
     static constexpr int W_LOAD = NSMW, W_MMA = NSMW + NLOAD;
     static constexpr int NT = (NSMW + NLOAD + 1) * 32;
     static constexpr uint32_t FULL_ARRIVALS = FP8 ? NLOAD * 32 : 1;  // arrivals that fill a K or V slot
-    // TMEM columns: S_t (and P_t in its first KT/2 columns) at t * KT; O_t at COL_O + t * D
+    // TMEM columns: S_t at t * KT (and for an E4M3 cache P_t in its first
+    // KT/2 columns); O_t at COL_O + t * D
     static constexpr uint32_t COL_O = NQ * KT;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TX_BYTES = KTILE;   // one K or V tile
@@ -116,24 +147,31 @@ struct PCfg {
     static_assert(COL_O + NQ * D <= TMEM_COLS, "TMEM columns");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(SCOL % 64 == 0 && OCOL % 32 == 0, "whole TMEM column groups per thread");
+    static_assert(!FP8 || NSK == NSV, "the E4M3 loader fills K and V slots in pairs");
+    static_assert(NSPLIT * 128 * 4 <= QTILE, "row sums fit in a query tile's buffer");
 };
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
     prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
-    constexpr int D = C::D, G = C::G, KT = C::KT, NS = C::NSLOT, NQ = C::NQ;
+    constexpr int D = C::D, G = C::G, KT = C::KT, NSK = C::NSK, NSV = C::NSV, NQ = C::NQ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *sQ = smem + C::OFF_Q;
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
+    uint8_t *sP = smem + C::OFF_P;  // P_t (bf16 cache): 128 rows x KT keys, 128-byte swizzle
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *kfull = bars, *kempty = bars + NS, *vfull = bars + 2 * NS, *vempty = bars + 3 * NS;
-    uint64_t *sfull = bars + 4 * NS, *pfull = sfull + NQ, *odone = pfull + NQ, *ofinal = odone + NQ;
-    uint64_t *mma_done = ofinal + NQ;
-    uint64_t *kload = mma_done + 1, *vload = kload + NS;  // E4M3: the codes of a tile have landed
+    uint64_t *kfull = bars, *kempty = kfull + NSK, *vfull = kempty + NSK, *vempty = vfull + NSV;
+    uint64_t *sfull = vempty + NSV, *pfull = sfull + NQ, *odone = pfull + NQ, *ofinal = odone + NQ;
+    uint64_t *sfree = ofinal + NQ;                       // P in shared memory: S_t has been read
+    uint64_t *mma_done = sfree + (C::PSMEM ? NQ : 0);
+    uint64_t *kload = mma_done + 1, *vload = kload + NSK;  // E4M3: the codes of a tile have landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
-    float *xch = reinterpret_cast<float *>(smem + C::OFF_X);  // [3][NQ][NSPLIT][128]: max (2 parities), sum
+    // [3][NQ][NSPLIT][128] fp32: max (2 parities), sum; with P in shared
+    // memory [2][NQ][NSPLIT][128] bf16 maxima
+    float *xch = reinterpret_cast<float *>(smem + C::OFF_X);
+    uint16_t *xch16 = reinterpret_cast<uint16_t *>(smem + C::OFF_X);
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     // CTA -> (chunk c, kv head, query tiles from i0).  CTAs start in the order
@@ -152,6 +190,10 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int i0 = qx * (NQ * C::QPOS);
     pdl_trigger();
     pdl_wait();
+    if (C::SLACK == 0 && smem != smem_raw) {  // no room to align: the base must be aligned (uniform per launch)
+        if (tid == 0) flag_error(a.err, PA_DEVERR_LAYOUT);
+        return;
+    }
     const uint64_t deadline = wait_deadline();  // shared by every wait of this launch
     // causal chunk: rows are positions pfx + i, keys [0, pfx + i]; shared
     // prefix: rows are sequences, keys [0, shared_len) for every row
@@ -188,17 +230,24 @@ __global__ void __launch_bounds__(C::NT, 1)
 
     if (w == C::W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 4 * NS; ++i)  // full barriers: [0, NS) and [2NS, 3NS)
-            mbar_init(&bars[i], (i < NS || (i >= 2 * NS && i < 3 * NS)) ? C::FULL_ARRIVALS : 1);
+        for (int i = 0; i < NSK; ++i) {
+            mbar_init(&kfull[i], C::FULL_ARRIVALS);
+            mbar_init(&kempty[i], 1);
+        }
+        for (int i = 0; i < NSV; ++i) {
+            mbar_init(&vfull[i], C::FULL_ARRIVALS);
+            mbar_init(&vempty[i], 1);
+        }
         for (int t = 0; t < NQ; ++t) {
             mbar_init(&sfull[t], 1);
             mbar_init(&pfull[t], 128 * C::NSPLIT);
             mbar_init(&odone[t], 1);
             mbar_init(&ofinal[t], 1);
+            if constexpr (C::PSMEM) mbar_init(&sfree[t], 128 * C::NSPLIT);
         }
         mbar_init(mma_done, 1);
         if constexpr (C::FP8)
-            for (int i = 0; i < 2 * NS; ++i) mbar_init(&kload[i], 1);
+            for (int i = 0; i < NSK + NSV; ++i) mbar_init(&kload[i], 1);
         fence_mbar_init();
     }
     // ---- query tiles: row r of tile t = (position r / G, head r % G), 128-byte swizzle.
@@ -296,6 +345,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         // the slot's full barrier.  A slot is refilled once the MMAs reading
         // its previous tile have completed (its empty barrier).
         constexpr int BPT = KT / 16;  // blocks per tile
+        constexpr int NS = C::NSK;    // K and V slots (as many of each)
         const int ct = tid - C::W_LOAD * 32;
         const bool issuer = w == C::W_LOAD;
         int win0 = jt0 * BPT, went = issuer ? bt[min(win0 + lane, nalloc - 1)] : 0;
@@ -385,66 +435,74 @@ __global__ void __launch_bounds__(C::NT, 1)
             __syncwarp();
         }
     } else if (!C::FP8 && w == C::W_LOAD) {
-        // ---- producer: K tile j, then V tile j, into ring slot j % NS.  The
-        // warp keeps a window of 32 block-table entries in registers (lane l
-        // holds entry win0 + l), refilled every 32/BPT tiles, so a tile's
-        // copies are issued without a global round trip.
+        // ---- producer: K tile j+1, then V tile j, into rings of NSK and NSV
+        // slots (K_{j+1} is needed by the next scores while tile j's softmax
+        // runs, V_j only by tile j's P.V).  The warp keeps a window of 32
+        // block-table entries in registers (lane l holds entry win0 + l),
+        // refilled every 32/BPT tiles, so a tile's copies are issued without
+        // a global round trip; a tile's row is kept from its K copy for its V.
         constexpr int BPT = KT / 16;  // blocks per tile
         int win0 = jt0 * BPT, went = bt[min(win0 + lane, nalloc - 1)];
-        int kissued = 0, vissued = 0;  // tiles whose K / V copies were issued
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % NS, jb = (jt0 + j) * BPT;  // first block of the tile
-            const uint32_t use = j / NS;  // how many times slot s was filled before
+        auto tile_row = [&](int jj) {  // lanes 0..BPT-1: cache row of block jj*BPT + lane (tiles in order)
+            const int jb = (jt0 + jj) * BPT;
             if (jb + BPT > win0 + 32) {
                 win0 = jb;
                 went = bt[min(win0 + lane, nalloc - 1)];
             }
-            // lanes 0..BPT-1: block jb + lane (past the end: the last block, masked later)
+            // past the end: the last block, masked later
             int phys = __shfl_sync(0xffffffffu, went, (min(jb + lane % BPT, nalloc - 1) - win0) & 31);
             if (lane < BPT && (phys < 0 || phys >= a.num_blocks)) {
                 flag_error(a.err, PA_DEVERR_BAD_BLOCK);
                 phys = 0;
             }
-            const int row = (phys * a.Hkv + kvh) * 16;
+            return (phys * a.Hkv + kvh) * 16;
+        };
+        int kissued = 0, vissued = 0;  // tiles whose K / V copies were issued
+        auto fill = [&](int jj, int kv, int row) {  // wait for the slot, then copy tile jj of K (kv 0) or V
+            const int ns = kv ? NSV : NSK, sl = jj % ns;
+            const uint32_t use = jj / ns;  // how many times the slot was filled before
+            if (use > 0 && !wait(kv ? &vempty[sl] : &kempty[sl], (use - 1) & 1)) return false;
+            (kv ? vissued : kissued) = jj + 1;
+            uint64_t *full = kv ? &vfull[sl] : &kfull[sl];
+            if (lane == 0) mbar_arrive_expect_tx(full, C::TX_BYTES);
+            __syncwarp();
+            if (lane < BPT) {
+                uint8_t *dst = (kv ? sV : sK) + sl * C::KTILE + lane * 16 * 128;
 #pragma unroll
-            for (int kv = 0; kv < 2; ++kv) {
-                uint64_t *full = kv ? &vfull[s] : &kfull[s];
-                if (use > 0 && !wait(kv ? &vempty[s] : &kempty[s], (use - 1) & 1)) break;
-                (kv ? vissued : kissued) = j + 1;
-                if (lane == 0) mbar_arrive_expect_tx(full, C::TX_BYTES);
-                __syncwarp();
-                if (lane < BPT) {
-                    uint8_t *dst = (kv ? sV : sK) + s * C::KTILE + lane * 16 * 128;
-#pragma unroll
-                    for (int at = 0; at < C::NATOM; ++at)
-                        tma_load_2d(dst + at * C::KATOM, kv ? &tmV : &tmK, at * 64, row, full);
-                }
-                __syncwarp();
+                for (int at = 0; at < C::NATOM; ++at)
+                    tma_load_2d(dst + at * C::KATOM, kv ? &tmV : &tmK, at * 64, row, full);
             }
+            __syncwarp();
+            return true;
+        };
+        int row_next = ntiles > 0 ? tile_row(0) : 0;
+        if (ntiles > 0) fill(0, 0, row_next);
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int row = row_next;
+            if (j + 1 < ntiles) {
+                row_next = tile_row(j + 1);
+                if (!fill(j + 1, 0, row_next)) break;
+            }
+            if (!fill(j, 1, row)) break;
         }
         if (!ok) {
             // each slot has at most one copy in flight (a slot is refilled only
             // after its previous fill was consumed): wait for the last fill of
             // every slot, with a short fresh budget
             const uint64_t dd = drain_deadline();
-            for (int sl = 0; sl < NS; ++sl) {
-                if (kissued > sl) mbar_wait(&kfull[sl], ((kissued - 1 - sl) / NS) & 1, dd);
-                if (vissued > sl) mbar_wait(&vfull[sl], ((vissued - 1 - sl) / NS) & 1, dd);
-            }
+            for (int sl = 0; sl < NSK; ++sl)
+                if (kissued > sl) mbar_wait(&kfull[sl], ((kissued - 1 - sl) / NSK) & 1, dd);
+            for (int sl = 0; sl < NSV; ++sl)
+                if (vissued > sl) mbar_wait(&vfull[sl], ((vissued - 1 - sl) / NSV) & 1, dd);
             __syncwarp();
         }
     } else if (w == C::W_MMA) {
-        // ---- MMA issue, software-pipelined per query tile: O_t += P_t(j) V_j
-        // as soon as softmax t hands over P_t(j), then S_t(j+1) = Q_t K_{j+1}^T
-        // as soon as that P.V has completed (S_t(j+1) overwrites P_t).  Tile
-        // 0's next scores never wait for tile 1's softmax, and tile 1 stays
-        // half a step behind tile 0, so the two softmaxes use MUFU in turns.
         constexpr uint32_t idS = idesc_f16kind_f32(128, KT, false, !C::FP8);
         constexpr uint32_t idO = idesc_f16kind_f32(128, D, true, !C::FP8);
-        auto issue_s = [&](int t, int jj) {
+        auto issue_s = [&](int t, int ks) {  // S_t from the K tile in ring slot ks
             if (lane == 0) {
                 tc_fence_after();
-                const uint32_t q0 = smem_addr(sQ + t * C::QTILE), k0 = smem_addr(sK + (jj % NS) * C::KTILE);
+                const uint32_t q0 = smem_addr(sQ + t * C::QTILE), k0 = smem_addr(sK + ks * C::KTILE);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     tc_mma_bf16(tmem + t * KT, smem_desc_sw128(q0 + (kk / 4) * C::QATOM + (kk % 4) * 32, 16, 1024),
@@ -453,20 +511,9 @@ __global__ void __launch_bounds__(C::NT, 1)
             }
             __syncwarp();
         };
-        if (ntiles > 0 && wait(&kfull[0], 0)) {
-#pragma unroll
-            for (int t = 0; t < NQ; ++t)
-                if (ntl[t] > 0) issue_s(t, 0);
-            if (lane == 0) tc_commit(&kempty[0]);
-            __syncwarp();
-        }
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % NS, jn = j + 1, sn = jn % NS;
-            if (!wait(&vfull[s], (j / NS) & 1)) break;
+        auto zero_tail = [&](int j, uint8_t *vt) {  // key rows past the sequence end: zero them before they meet P
             const int kv0 = (jt0 + j) * KT;
-            if (!C::FP8 && kv0 + KT > L) {  // key rows past the sequence end: zero them before they meet P
-                // (the converters of an E4M3 cache write those rows as zeros)
-                uint8_t *vt = sV + s * C::KTILE;
+            if (!C::FP8 && kv0 + KT > L) {  // (the loader of an E4M3 cache writes those rows as zeros)
                 for (int r = max(L - kv0, 0) + lane; r < KT; r += 32)
 #pragma unroll
                     for (int at = 0; at < C::NATOM; ++at)
@@ -476,40 +523,106 @@ __global__ void __launch_bounds__(C::NT, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            bool kready = false;  // K tile j+1 has landed
+        };
+        if (ntiles > 0 && wait(&kfull[0], 0)) {
 #pragma unroll
-            for (int t = 0; t < NQ; ++t) {
-                if (j < ntl[t]) {
-                    if (!wait(&pfull[t], j & 1)) break;  // P_t(j) is in TMEM
-                    if (lane == 0) {
-                        tc_fence_after();
-                        const uint32_t v0 = smem_addr(sV + s * C::KTILE);
+            for (int t = 0; t < NQ; ++t)
+                if (ntl[t] > 0) issue_s(t, 0);
+            if (lane == 0) tc_commit(&kempty[0]);
+            __syncwarp();
+        }
+        if constexpr (C::PSMEM) {
+            // ---- MMA issue with P in shared memory, per K/V tile j: first the
+            // next scores S_t(j+1) = Q_t K_{j+1}^T, each as soon as softmax t has
+            // loaded S_t(j) (S free); then O_t += P_t(j) V_j as P_t(j) arrives
+            // The tensor core computes tile j+1's scores while tile j's
+            // exponentials run.
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int jn = j + 1;
+                if (jn < ntiles) {
+                    const int sn = jn % NSK;
+                    if (!wait(&kfull[sn], (jn / NSK) & 1)) break;
 #pragma unroll
-                        for (int kk = 0; kk < KT / 16; ++kk)
-                            tc_mma_bf16_tmem_a(tmem + C::COL_O + t * D, tmem + t * KT + kk * 8,
-                                               smem_desc_sw128(v0 + kk * 16 * 128, C::KATOM, 1024), idO,
-                                               j > 0 || kk > 0);
-                        tc_commit(&odone[t]);
-                        if (j == ntl[t] - 1) tc_commit(&ofinal[t]);
-                    }
+                    for (int t = 0; t < NQ; ++t)
+                        if (jn < ntl[t]) {
+                            if (!wait(&sfree[t], j & 1)) break;  // S_t(j) is in softmax t's registers
+                            issue_s(t, sn);
+                        }
+                    if (!ok) break;
+                    if (lane == 0) tc_commit(&kempty[sn]);  // after both S(j+1)
                     __syncwarp();
                 }
-                if (jn < ntl[t]) {
-                    if (!kready) {
-                        if (!wait(&kfull[sn], (jn / NS) & 1)) break;
-                        kready = true;
+                const int s = j % NSV;
+                if (!wait(&vfull[s], (j / NSV) & 1)) break;
+                zero_tail(j, sV + s * C::KTILE);
+#pragma unroll
+                for (int t = 0; t < NQ; ++t)
+                    if (j < ntl[t]) {
+                        if (!wait(&pfull[t], j & 1)) break;  // P_t(j) is in shared memory
+                        if (lane == 0) {
+                            tc_fence_after();
+                            const uint32_t p0 = smem_addr(sP + t * C::PTILE), v0 = smem_addr(sV + s * C::KTILE);
+#pragma unroll
+                            for (int kk = 0; kk < KT / 16; ++kk)
+                                tc_mma_bf16(tmem + C::COL_O + t * D,
+                                            smem_desc_sw128(p0 + (kk / 4) * C::PATOM + (kk % 4) * 32, 16, 1024),
+                                            smem_desc_sw128(v0 + kk * 16 * 128, C::KATOM, 1024), idO, j > 0 || kk > 0);
+                            tc_commit(&odone[t]);
+                            if (j == ntl[t] - 1) tc_commit(&ofinal[t]);
+                        }
+                        __syncwarp();
                     }
-                    if (!wait(&odone[t], j & 1)) break;  // P_t(j) consumed
-                    issue_s(t, jn);
-                }
-            }
-            if (!ok) break;
-            if (lane == 0) tc_commit(&vempty[s]);
-            __syncwarp();
-            if (jn < ntiles) {
-                if (!kready && !wait(&kfull[sn], (jn / NS) & 1)) break;
-                if (lane == 0) tc_commit(&kempty[sn]);  // after every S(j+1) above
+                if (!ok) break;
+                if (lane == 0) tc_commit(&vempty[s]);
                 __syncwarp();
+            }
+        } else {
+            // ---- MMA issue with P in TMEM (E4M3 cache), software-pipelined
+            // per query tile: O_t += P_t(j) V_j as soon as softmax t hands over
+            // P_t(j), then S_t(j+1) = Q_t K_{j+1}^T as soon as that P.V has
+            // completed (S_t(j+1) overwrites P_t).  Tile 0's next scores never
+            // wait for tile 1's softmax, and tile 1 stays half a step behind
+            // tile 0, so the two softmaxes use MUFU in turns.
+            constexpr int NS = NSK;
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int s = j % NS, jn = j + 1, sn = jn % NS;
+                if (!wait(&vfull[s], (j / NS) & 1)) break;
+                zero_tail(j, sV + s * C::KTILE);
+                bool kready = false;  // K tile j+1 has landed
+#pragma unroll
+                for (int t = 0; t < NQ; ++t) {
+                    if (j < ntl[t]) {
+                        if (!wait(&pfull[t], j & 1)) break;  // P_t(j) is in TMEM
+                        if (lane == 0) {
+                            tc_fence_after();
+                            const uint32_t v0 = smem_addr(sV + s * C::KTILE);
+#pragma unroll
+                            for (int kk = 0; kk < KT / 16; ++kk)
+                                tc_mma_bf16_tmem_a(tmem + C::COL_O + t * D, tmem + t * KT + kk * 8,
+                                                   smem_desc_sw128(v0 + kk * 16 * 128, C::KATOM, 1024), idO,
+                                                   j > 0 || kk > 0);
+                            tc_commit(&odone[t]);
+                            if (j == ntl[t] - 1) tc_commit(&ofinal[t]);
+                        }
+                        __syncwarp();
+                    }
+                    if (jn < ntl[t]) {
+                        if (!kready) {
+                            if (!wait(&kfull[sn], (jn / NS) & 1)) break;
+                            kready = true;
+                        }
+                        if (!wait(&odone[t], j & 1)) break;  // P_t(j) consumed
+                        issue_s(t, sn);
+                    }
+                }
+                if (!ok) break;
+                if (lane == 0) tc_commit(&vempty[s]);
+                __syncwarp();
+                if (jn < ntiles) {
+                    if (!kready && !wait(&kfull[sn], (jn / NS) & 1)) break;
+                    if (lane == 0) tc_commit(&kempty[sn]);  // after every S(j+1) above
+                    __syncwarp();
+                }
             }
         }
         // every MMA of this CTA has completed before TMEM is released (after
@@ -556,6 +669,10 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
                 for (int e = 0; e < SCOL; ++e) sv[e] = -INFINITY;
             }
+            if constexpr (C::PSMEM) {  // S_t(j) is in registers: the next scores may overwrite it
+                tc_fence_before();
+                mbar_arrive(&sfree[t]);
+            }
             // raw scores (the scale is positive, so the max commutes with it);
             // the causal mask only where the tile reaches past this row
             const int kv0 = (jt0 + j) * KT + half * SCOL;
@@ -568,10 +685,21 @@ __global__ void __launch_bounds__(C::NT, 1)
             for (int e = 0; e < SCOL; e += 2) mraw = fmax3(mraw, sv[e], sv[e + 1]);
             // the row's max over its threads; after this barrier every thread
             // of the row has read its S columns, so P may overwrite them
-            *xslot(j & 1, half) = mraw;
-            named_bar_sync(bar_id, 32 * NSP);
+            if constexpr (C::PSMEM) {
+                // as bf16 rounded up: every thread of the row takes the max of
+                // the same rounded values, and it stays >= the true row max
+                uint16_t *x = xch16 + ((j & 1) * NQ + t) * NSP * 128 + r;
+                x[half * 128] = __bfloat16_as_ushort(__float2bfloat16_ru(mraw));
+                named_bar_sync(bar_id, 32 * NSP);
+                mraw = -INFINITY;
 #pragma unroll
-            for (int hh = 0; hh < NSP; ++hh) mraw = fmaxf(mraw, *xslot(j & 1, hh));
+                for (int hh = 0; hh < NSP; ++hh) mraw = fmaxf(mraw, __uint_as_float((uint32_t)x[hh * 128] << 16));
+            } else {
+                *xslot(j & 1, half) = mraw;
+                named_bar_sync(bar_id, 32 * NSP);
+#pragma unroll
+                for (int hh = 0; hh < NSP; ++hh) mraw = fmaxf(mraw, *xslot(j & 1, hh));
+            }
             if (!ok) {
                 mbar_arrive(&pfull[t]);
                 continue;
@@ -589,6 +717,7 @@ __global__ void __launch_bounds__(C::NT, 1)
             const float mb = (m == -INFINITY) ? 0.f : m;
             const float2 sc2 = make_float2(sl2, sl2), nb2 = make_float2(-mb, -mb);
             float2 sum2 = make_float2(0.f, 0.f);
+            bool ready = true;  // P in shared memory: P_t(j-1).V_{j-1} has completed
 #pragma unroll
             for (int h = 0; h < SCOL / 64; ++h) {
                 uint32_t pk[32];
@@ -617,13 +746,28 @@ __global__ void __launch_bounds__(C::NT, 1)
                                                        __uint_as_float((wh >> 16) << 13)));
                     }
                 }
-                tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
+                if constexpr (C::PSMEM) {
+                    // P_t(j) goes where P_t(j-1) was, once its P.V has read it
+                    // (that also makes O_t complete up to tile j-1)
+                    if (h == 0 && j > 0) ready = wait_all(&odone[t], (j - 1) & 1);
+                    if (ready) {
+                        uint8_t *prow = sP + t * C::PTILE + ((half * SCOL) / 64 + h) * C::PATOM + r * 128;
+#pragma unroll
+                        for (int cc = 0; cc < 8; ++cc)
+                            *reinterpret_cast<uint4 *>(prow + ((cc ^ (r & 7)) * 16)) =
+                                make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+                    }
+                } else {
+                    tmem_st32_u(lane_base + pcol + 32 * h, pk);  // P over S columns already read
+                }
             }
             l += sum2.x + sum2.y;  // this thread's keys; the row sum is combined at the end
-            // O_t holds P.V up to tile j-1, complete (S_t(j) was issued after it):
-            // rescale in TMEM; tcgen05.ld/st are warp-collective, so the warp
-            // rescales if any of its rows needs it
-            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+            // O_t holds P.V up to tile j-1, complete (P in shared memory: the
+            // wait above; else S_t(j) was issued after it): rescale in TMEM;
+            // tcgen05.ld/st are warp-collective, so the warp rescales if any of
+            // its rows needs it
+            if (C::PSMEM) tc_fence_after();
+            if (ready && j > 0 && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                 for (int q = 0; q < OCOL / 32; ++q) {
                     float o[32];
@@ -634,19 +778,34 @@ __global__ void __launch_bounds__(C::NT, 1)
                     tmem_st32(lane_base + ocol + 32 * q, o);
                 }
             }
+            if constexpr (C::PSMEM) fence_proxy_async_smem();  // P stores -> the tensor core
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&pfull[t]);
         }
         if (ntl[t] > 0) {
-            // ---- epilogue: O / l, as bf16 output rows (or as split-K piece kz)
-            *xslot(2, half) = l;
-            named_bar_sync(bar_id, 32 * NSP);
-            l = 0.f;
+            // ---- epilogue: O / l, as bf16 output rows (or as split-K piece kz).
+            // The row sum over its threads: with P in shared memory through
+            // Q_t's buffer, which is free once O_t is final
+            bool fin;
+            if constexpr (C::PSMEM) {
+                fin = wait_all(&ofinal[t], 0);
+                float *xs = reinterpret_cast<float *>(sQ + t * C::QTILE) + r;
+                xs[half * 128] = l;
+                named_bar_sync(bar_id, 32 * NSP);
+                l = 0.f;
 #pragma unroll
-            for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
-            if constexpr (C::FP8) l *= 0x1p112f;  // the f16 sum was kept scaled by 2^-112
-            if (wait_all(&ofinal[t], 0)) {
+                for (int hh = 0; hh < NSP; ++hh) l += xs[hh * 128];
+            } else {
+                *xslot(2, half) = l;
+                named_bar_sync(bar_id, 32 * NSP);
+                l = 0.f;
+#pragma unroll
+                for (int hh = 0; hh < NSP; ++hh) l += *xslot(2, hh);
+                if constexpr (C::FP8) l *= 0x1p112f;  // the f16 sum was kept scaled by 2^-112
+                fin = wait_all(&ofinal[t], 0);
+            }
+            if (fin) {
                 tc_fence_after();
                 const size_t grow = (size_t)(q_start + ip) * a.Hq + (size_t)kvh * G + r % G;  // q / out row
                 __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + grow * D + half * OCOL;

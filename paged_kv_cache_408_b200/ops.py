@@ -21,6 +21,7 @@ PA_OK = 0
 DTYPE_BF16, DTYPE_FP8_E4M3 = 0, 1
 
 DEVERR_BAD_BLOCK, DEVERR_BAD_SLOT, DEVERR_BAD_LEN, DEVERR_BAD_PAIR, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
+DEVERR_LAYOUT = 0x20
 
 EXPORTED = (
     "pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_size", "pa_decode", "pa_prefill_chunk",

@@ -55,11 +55,26 @@ def run_decode(case, kc, vc, seq_lens=None, partition_tokens=0, block_tables=Non
     return out
 
 
+def bf16_step(x):
+    """Spacing of bf16 values at magnitude |x| (2^(e-7) for |x| in [2^e, 2^(e+1)))."""
+    return np.exp2(np.floor(np.log2(np.maximum(np.abs(x), 1e-300))) - 7)
+
+
 def assert_attn_close(got, ref, what=""):
+    """The attention tolerance: every element within max-abs 1e-2 of the
+    fp64 result, or -- where one bf16 step exceeds that (|x| >= 2, rows
+    carried by one or two keys) -- less than one bf16 step from it (the
+    kernel's fp32 result may lie on the other side of a rounding midpoint);
+    mean-abs over all elements <= 1e-3."""
     err = np.abs(got - ref)
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
-    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}"
+    bad = (err > MAX_ABS) & (err >= bf16_step(np.maximum(np.abs(got), np.abs(ref))))
+    if bad.any() or not mean <= MEAN_ABS:
+        at = np.unravel_index(int(np.argmax(np.where(bad, err, 0.0) if bad.any() else err)), err.shape)
+        raise AssertionError(f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}; worst at {tuple(int(i) for i in at)}: "
+                             f"got {float(got[at]):.6f}, expected {float(ref[at]):.6f}; "
+                             f"{int(bad.sum())} of {err.size} beyond the tolerance")
     return mx, mean
 
 
@@ -83,8 +98,7 @@ def assert_attn_close_bf16(got, exact, what=""):
     err = np.abs(got - exact)
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     mag = np.maximum(np.abs(got), np.abs(exact))
-    step = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-300))) - 7)  # bf16 spacing at that magnitude
-    bad = ~((err <= MAX_ABS) | (err < step))
+    bad = ~((err <= MAX_ABS) | (err < bf16_step(mag)))
     assert not bad.any(), f"{what}: {int(bad.sum())} outputs off by more than max-abs and one bf16 step, " \
                           f"worst {float(err[bad].max()):.3e}"
     mean = float(np.abs(got - bf16_round(exact)).mean())

@@ -14,7 +14,18 @@ Checked for every schedule: no deadlock; no waiter sees its barrier two or
 more phases past the one it waits for (a parity wait would pass on a stale
 phase); S_t(j+1) is never issued before P_t(j).V_j has completed.  Two planted
 protocol mistakes (an O-done wait skipped on odd tiles, S issued without the
-O-done wait) must each be caught."""
+O-done wait) must each be caught.
+
+With a bf16 cache the kernel keeps P in shared memory instead (`psmem`
+below): the loader fills K_{j+1} before V_j into a K ring and a V ring;
+the MMA warp issues S_t(j+1) as soon as softmax t has loaded S_t(j) into
+registers ("S free") and then P_t(j).V_j once P_t(j) is in shared memory;
+softmax t writes P_t(j) only after P_t(j-1).V_{j-1} has
+completed (O done), which also makes its O rescale safe.  Checked: the
+softmax always reads the scores of the tile it waits for, every MMA reads
+the K or V tile it expects, P_t(j) is still in its buffer when its P.V
+completes, a slot is never refilled before the MMAs reading it completed.
+Planted: the S-free wait skipped, the O-done wait before the P write skipped."""
 import random
 
 import pytest
@@ -195,6 +206,175 @@ def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False, fp8=Fa
     return None
 
 
+def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
+    """Random schedules of the P-in-shared-memory protocol (a K ring of nsk
+    slots, a V ring of nsv slots, a P buffer per query tile); None or the
+    first violation."""
+    nq, ntiles = len(ntl), max(ntl)
+    for seed in range(seeds):
+        rnd = random.Random(7000 + seed)
+        ns = {"k": nsk, "v": nsv}
+        ring = {k + e: [Barrier(f"{k}{e}{i}") for i in range(ns[k])] for k in ("k", "v") for e in ("full", "empty")}
+        tile = {k: [Barrier(f"{k}{t}") for t in range(nq)] for k in ("sfull", "sfree", "pfull", "odone", "ofinal")}
+        consumed = {"k": [-1] * nsk, "v": [-1] * nsv}  # last tile whose MMAs completed, per slot
+        held = {"k": [-1] * nsk, "v": [-1] * nsv}      # the tile whose data sits in each slot
+        s_data = [-1] * nq   # the key tile whose scores sit in S_t's TMEM columns
+        p_data = [-1] * nq   # the key tile whose P sits in P_t's buffer
+        pv_done = [-1] * nq
+        pending, violation = [], []
+
+        class Done:  # an asynchronous completion: apply its effect, then arrive
+            def __init__(self, bar, effect=None):
+                self.bar, self.effect = bar, effect
+
+            def arrive(self):
+                if self.effect:
+                    self.effect()
+                self.bar.arrive()
+
+        def landed(kind, j):
+            def f():
+                held[kind][j % ns[kind]] = j
+            return f
+
+        def fill(kind, j):
+            sl, use = j % ns[kind], j // ns[kind]
+            if use:
+                yield ring[kind + "empty"][sl], use - 1
+                if consumed[kind][sl] < j - ns[kind]:
+                    yield None, f"{kind} tile {j} copied over tile {j - ns[kind]} still in use"
+            pending.append(Done(ring[kind + "full"][sl], landed(kind, j)))
+
+        def loader():
+            if ntiles:
+                yield from fill("k", 0)
+            for j in range(ntiles):
+                if j + 1 < ntiles:
+                    yield from fill("k", j + 1)
+                yield from fill("v", j)
+
+        def consumed_by(kind, sl, j):
+            def f():
+                consumed[kind][sl] = max(consumed[kind][sl], j)
+            return f
+
+        def scores(t, j):
+            def f():
+                if held["k"][j % nsk] != j:
+                    violation.append(f"S_{t}({j}) computed from K tile {held['k'][j % nsk]}")
+                s_data[t] = j
+            return f
+
+        def pv(t, j):
+            def f():
+                if p_data[t] != j:
+                    violation.append(f"P_{t}({j}).V completed with P_{t}({p_data[t]}) in the buffer")
+                if held["v"][j % nsv] != j:
+                    violation.append(f"P_{t}({j}).V read V tile {held['v'][j % nsv]}")
+                pv_done[t] = j
+            return f
+
+        def mma():
+            if ntiles:
+                yield ring["kfull"][0], 0
+                for t in range(nq):
+                    if ntl[t]:
+                        pending.append(Done(tile["sfull"][t], scores(t, 0)))
+                pending.append(Done(ring["kempty"][0], consumed_by("k", 0, 0)))
+            for j in range(ntiles):
+                jn = j + 1
+                if jn < ntiles:
+                    sn = jn % nsk
+                    yield ring["kfull"][sn], jn // nsk
+                    for t in range(nq):
+                        if jn < ntl[t]:
+                            if not skip_sfree:
+                                yield tile["sfree"][t], j
+                            pending.append(Done(tile["sfull"][t], scores(t, jn)))
+                    pending.append(Done(ring["kempty"][sn], consumed_by("k", sn, jn)))
+                sv = j % nsv
+                yield ring["vfull"][sv], j // nsv
+                for t in range(nq):
+                    if j < ntl[t]:
+                        yield tile["pfull"][t], j
+                        pending.append(Done(tile["odone"][t], pv(t, j)))
+                        if j == ntl[t] - 1:
+                            pending.append(Done(tile["ofinal"][t]))
+                pending.append(Done(ring["vempty"][sv], consumed_by("v", sv, j)))
+                if violation:
+                    yield None, violation[0]
+
+        def softmax(t):
+            for j in range(ntl[t]):
+                yield tile["sfull"][t], j
+                if s_data[t] != j:
+                    yield None, f"softmax {t} read the scores of tile {s_data[t]} for tile {j}"
+                tile["sfree"][t].arrive()
+                if j > 0:
+                    if not skip_odone:
+                        yield tile["odone"][t], j - 1
+                    if pv_done[t] < j - 1:
+                        yield None, f"P_{t}({j}) written (and O_{t} rescaled) before P_{t}({j - 1}).V completed"
+                p_data[t] = j
+                tile["pfull"][t].arrive()
+            if ntl[t]:
+                yield tile["ofinal"][t], 0
+                if pv_done[t] != ntl[t] - 1:
+                    yield None, f"epilogue of tile {t} before its last P.V"
+
+        actors = {"load": loader(), "mma": mma(), **{f"softmax{t}": softmax(t) for t in range(nq)}}
+        err = run_schedule(actors, pending, rnd)
+        if err or violation:
+            return f"seed {seed}: {err or violation[0]}"
+    return None
+
+
+def run_schedule(actors, pending, rnd):
+    """Drive generator actors that yield (barrier, phase) waits, or (None,
+    message) for a violation; completions in `pending` arrive in order at
+    random times, and an actor that could run is delayed now and then (so a
+    completion may overtake a thread between its wait and its next step).
+    Returns None or the first violation / deadlock."""
+    waiting = {k: None for k in actors}
+    done = set()
+    while len(done) < len(actors):
+        progress = False
+        if pending and rnd.random() < 0.5:
+            pending.pop(0).arrive()
+            progress = True
+        order = list(actors)
+        rnd.shuffle(order)
+        for k in order:
+            if k in done:
+                continue
+            if waiting[k] is not None:
+                bar, phase = waiting[k]
+                if bar is None:
+                    return phase
+                if bar.phase > phase + 1:
+                    return f"{k} waits for phase {phase} of {bar.name}, already at {bar.phase}"
+                if bar.phase <= phase:
+                    continue
+            if rnd.random() < 0.3:  # runnable, but slow this round
+                progress = True
+                continue
+            waiting[k] = None
+            try:
+                waiting[k] = next(actors[k])
+                if waiting[k][0] is None:
+                    return waiting[k][1]
+            except StopIteration:
+                done.add(k)
+            progress = True
+        if not progress:
+            if pending:
+                pending.pop(0).arrive()
+                continue
+            stuck = {k: (w[0].name, w[1]) for k, w in waiting.items() if w and k not in done}
+            return f"deadlock {stuck}"
+    return None
+
+
 # (K/V tiles of query tile 0, of query tile 1): a causal chunk's second tile
 # needs one more key tile; a tile past the chunk end needs none
 SHAPES = [(1, 0), (3, 0), (2, 3), (5, 6), (9, 10), (1, 1), (4, 4), (8, 8)]
@@ -204,6 +384,26 @@ SHAPES = [(1, 0), (3, 0), (2, 3), (5, 6), (9, 10), (1, 1), (4, 4), (8, 8)]
 @pytest.mark.parametrize("nslot", [2, 4])
 def test_protocol_has_no_deadlock_aliasing_or_overwrite(ntl, nslot):
     assert explore(list(ntl), nslot, seeds=120) is None
+
+
+@pytest.mark.parametrize("ntl", SHAPES)
+@pytest.mark.parametrize("nsk,nsv", [(2, 1), (3, 3), (1, 1)])
+def test_psmem_protocol_has_no_deadlock_stale_data_or_overwrite(ntl, nsk, nsv):
+    """P in shared memory (bf16 cache): 2 K slots and 1 V slot at head_dim
+    128, 3 and 3 at head_dim 64, a P buffer per query tile."""
+    assert explore_psmem(list(ntl), nsk, nsv, seeds=120) is None
+
+
+def test_psmem_skipped_s_free_wait_is_caught():
+    found = [explore_psmem([6, 7], 2, 1, seeds=200, skip_sfree=True),
+             explore_psmem([9, 10], 3, 3, seeds=200, skip_sfree=True)]
+    assert all(found), found
+
+
+def test_psmem_p_written_before_its_buffer_is_free_is_caught():
+    found = [explore_psmem([6, 7], 2, 1, seeds=200, skip_odone=True),
+             explore_psmem([9, 10], 3, 3, seeds=200, skip_odone=True)]
+    assert all(found), found
 
 
 @pytest.mark.parametrize("ntl", SHAPES)
@@ -249,13 +449,16 @@ def test_issuing_s_without_the_o_done_wait_is_caught():
 # finishes (no thread stranded at a named barrier), and no actor issues a
 # protocol wait after its first failed one.
 
-def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_failure=False):
+def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_failure=False, psmem=None):
+    """psmem = (nsk, nsv): the P-in-shared-memory protocol of a bf16 cache."""
     nq, ntiles = len(ntl), max(ntl)
+    nsk, nsv = psmem if psmem else (nslot, nslot)
     for seed in range(seeds):
         rnd = random.Random(1000 + seed)
-        ring = {k: [Barrier(f"{k}{i}") for i in range(nslot)] for k in ("kfull", "kempty", "vfull", "vempty")}
-        tile = {k: [Barrier(f"{k}{t}", 2 if k == "pfull" else 1) for t in range(nq)]
-                for k in ("sfull", "pfull", "odone", "ofinal")}
+        ring = {k: [Barrier(f"{k}{i}") for i in range(nsk if k[0] == "k" else nsv)]
+                for k in ("kfull", "kempty", "vfull", "vempty")}
+        tile = {k: [Barrier(f"{k}{t}", 2 if k in ("pfull", "sfree") else 1) for t in range(nq)]
+                for k in ("sfull", "sfree", "pfull", "odone", "ofinal")}
         mma_done = Barrier("mma_done")
         pending = []
         drop_at = rnd.randrange(1, 4 * ntiles * (nq + 2) + 2)
@@ -351,8 +554,97 @@ def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_fail
                 yield ("named", t)
                 ok = yield from wait(tile["ofinal"][t], 0, ok)
 
-        actors = {"load": loader(), "mma": mma(),
-                  **{f"softmax{t}.{h}": softmax(t, h) for t in range(nq) for h in range(2)}}
+        def loader_ps():
+            ok, issued = True, {"k": 0, "v": 0}
+            ns = {"k": nsk, "v": nsv}
+
+            def fill(kind, j, ok):
+                sl, use = j % ns[kind], j // ns[kind]
+                if use:
+                    ok = yield from wait(ring[kind + "empty"][sl], use - 1, ok)
+                    if not ok:
+                        return False
+                issued[kind] = j + 1
+                post(ring[kind + "full"][sl])
+                return True
+
+            if ntiles:
+                ok = yield from fill("k", 0, ok)
+            for j in range(ntiles):
+                if not ok:
+                    break
+                if j + 1 < ntiles:
+                    ok = yield from fill("k", j + 1, ok)
+                    if not ok:
+                        break
+                ok = yield from fill("v", j, ok)
+            if not ok:
+                for kind in ("k", "v"):
+                    for sl in range(ns[kind]):
+                        if issued[kind] > sl:
+                            yield ("drain", ring[kind + "full"][sl], (issued[kind] - 1 - sl) // ns[kind])
+
+        def mma_ps():
+            ok = True
+            if ntiles:
+                ok = yield from wait(ring["kfull"][0], 0, ok)
+                if ok:
+                    for t in range(nq):
+                        if ntl[t]:
+                            post(tile["sfull"][t])
+                    post(ring["kempty"][0])
+            for j in range(ntiles):
+                if not ok:
+                    break
+                jn = j + 1
+                if jn < ntiles:
+                    ok = yield from wait(ring["kfull"][jn % nsk], jn // nsk, ok)
+                    for t in range(nq):
+                        if ok and jn < ntl[t]:
+                            ok = yield from wait(tile["sfree"][t], j, ok)
+                            if ok:
+                                post(tile["sfull"][t])
+                    if not ok:
+                        break
+                    post(ring["kempty"][jn % nsk])
+                ok = yield from wait(ring["vfull"][j % nsv], j // nsv, ok)
+                for t in range(nq):
+                    if ok and j < ntl[t]:
+                        ok = yield from wait(tile["pfull"][t], j, ok)
+                        if ok:
+                            post(tile["odone"][t])
+                            if j == ntl[t] - 1:
+                                post(tile["ofinal"][t])
+                if not ok:
+                    break
+                post(ring["vempty"][j % nsv])
+            post(mma_done)
+            yield ("wait" if ok else "drain", mma_done, 0)
+
+        def softmax_ps(t, half):
+            ok = True
+            for j in range(ntl[t]):
+                ok = yield from wait(tile["sfull"][t], j, ok)
+                if not ok and break_softmax_loop:
+                    break
+                tile["sfree"][t].arrive()
+                yield ("named", t)
+                if not ok:
+                    tile["pfull"][t].arrive()
+                    continue
+                if j > 0:
+                    ok = yield from wait(tile["odone"][t], j - 1, ok)
+                tile["pfull"][t].arrive()
+            if ntl[t]:
+                ok = yield from wait(tile["ofinal"][t], 0, ok)
+                yield ("named", t)
+
+        if psmem:
+            actors = {"load": loader_ps(), "mma": mma_ps(),
+                      **{f"softmax{t}.{h}": softmax_ps(t, h) for t in range(nq) for h in range(2)}}
+        else:
+            actors = {"load": loader(), "mma": mma(),
+                      **{f"softmax{t}.{h}": softmax(t, h) for t in range(nq) for h in range(2)}}
         state = {k: None for k in actors}   # the event the actor is blocked on
         reply = {k: None for k in actors}
         failed = set()
@@ -424,6 +716,22 @@ def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_fail
 @pytest.mark.parametrize("nslot", [2, 4])
 def test_a_lost_transaction_ends_every_role_without_further_waits(ntl, nslot):
     assert explore_give_up(list(ntl), nslot, seeds=150) is None
+
+
+@pytest.mark.parametrize("ntl", [(1, 0), (3, 3), (5, 6), (9, 10)])
+@pytest.mark.parametrize("psmem", [(2, 1), (3, 3)])
+def test_psmem_lost_transaction_ends_every_role_without_further_waits(ntl, psmem):
+    assert explore_give_up(list(ntl), 0, seeds=150, psmem=psmem) is None
+
+
+def test_psmem_softmax_leaving_its_loop_after_a_failure_is_caught():
+    found = [explore_give_up([5, 6], 0, seeds=300, break_softmax_loop=True, psmem=ps) for ps in ((2, 1), (3, 3))]
+    assert any(f and "stranded" in f for f in found), found
+
+
+def test_psmem_waiting_again_after_a_failure_is_caught():
+    found = [explore_give_up([5, 6], 0, seeds=300, wait_after_failure=True, psmem=ps) for ps in ((2, 1), (3, 3))]
+    assert any(f and "after a failed one" in f for f in found), found
 
 
 def test_softmax_leaving_its_loop_after_a_failure_is_caught():
