@@ -165,3 +165,12 @@ def test_block_table_width_is_bounded():
                               C.byref(desc()), None) == -1
     assert L.pa_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, big, 32, 0.1, None, None, 0,
                                C.byref(desc()), None) == -1
+
+
+def test_device_status_bits_match_the_header():
+    """The binding's PA_DEVERR_* bits are the header's."""
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    bits = {m.group(1): int(m.group(2), 16) for m in re.finditer(r"#define PA_DEVERR_(\w+) (0x[0-9a-fA-F]+)u", text)}
+    assert bits == {"BAD_BLOCK": ops.DEVERR_BAD_BLOCK, "BAD_SLOT": ops.DEVERR_BAD_SLOT, "BAD_LEN": ops.DEVERR_BAD_LEN,
+                    "BAD_PAIR": ops.DEVERR_BAD_PAIR, "TIMEOUT": ops.DEVERR_TIMEOUT, "LAYOUT": ops.DEVERR_LAYOUT}
+    assert len(set(bits.values())) == len(bits) and all(b & (b - 1) == 0 for b in bits.values())
