@@ -355,46 +355,92 @@ def run_ours(args, rank, world, device, workload=None, legs_only=False):
     algf = [decode_alg_flops(ds.plan.decode_lens, Hq, D) for ds in timed if ds.B]
     launches = sum(e[3] for e in step_ev)
 
-    # ---- end to end: per-step inputs from pinned host memory, results read back
+    # ---- end to end: per-step inputs from pinned host memory, results read back.
+    # A serving loop's overlap: while step k runs, one copy stream brings step
+    # k+1's inputs in and another reads step k-1's outputs back (double
+    # buffers).  Step k's events end only once both have finished, so every
+    # copy lies inside some step's events: step k's time = max(its kernels,
+    # the copy of step k+1's inputs, the read of step k-1's outputs); step 0
+    # also covers its own inputs' copy, the last step its own read-back.
     e2e = None
     if not args.no_e2e:
         hsteps = [DeviceStep(p, torch, device, pin=True, cascade=not args.no_cascade) for p in plans[args.warmup:]]
         hq, hk, hv = q.cpu().pin_memory(), new_k.cpu().pin_memory(), new_v.cpu().pin_memory()
         hpq = pq.cpu().pin_memory()
         hout, hpout = torch.empty_like(hq).pin_memory(), torch.empty_like(hpq).pin_memory()
-        dq, dk, dv, dpq = torch.empty_like(q), torch.empty_like(new_k), torch.empty_like(new_v), torch.empty_like(pq)
+        dbuf = [(torch.empty_like(q), torch.empty_like(new_k), torch.empty_like(new_v), torch.empty_like(pq),
+                 torch.empty_like(out), torch.empty_like(pout)) for _ in range(2)]
+        cs_in, cs_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+        n = len(hsteps)
+        # device buffers allocated before timing (an allocation inside the
+        # loop could synchronise the device)
+        dmeta = [torch.empty(hs.nbytes(), dtype=torch.uint8, device=device) for hs in hsteps]
         ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in hsteps]
-        h2d = d2h = 0
+        landed, ran, read = ([torch.cuda.Event() for _ in hsteps] for _ in range(3))
+        dsteps_e2e = [None] * n
+        nbytes = {"h2d": 0, "d2h": 0}
+
+        def n_pf(hs):
+            return hs.n_prefill * Hq * D * 2 if attend_prefill else 0
+
+        def bring_in(k, after):  # step k's inputs, on the input copy stream, once `after` is reached
+            hs = hsteps[k]
+            cs_in.wait_event(after)
+            with torch.cuda.stream(cs_in):
+                dsteps_e2e[k] = hs.to(device, out=dmeta[k])
+                dq, dk, dv, dpq = dbuf[k % 2][:4]
+                if hs.B:
+                    dq[:hs.B].copy_(hq[:hs.B], non_blocking=True)
+                if hs.T:
+                    dk[:hs.T].copy_(hk[:hs.T], non_blocking=True)
+                    dv[:hs.T].copy_(hv[:hs.T], non_blocking=True)
+                if n_pf(hs):
+                    dpq[:hs.n_prefill].copy_(hpq[:hs.n_prefill], non_blocking=True)
+                landed[k].record(cs_in)
+            nbytes["h2d"] += hs.nbytes() + hs.B * Hq * D * 2 + 2 * hs.T * Hkv * D * 2 + n_pf(hs)
+
+        def read_back(k, stream, after):  # step k's outputs to pinned host memory
+            hs = hsteps[k]
+            stream.wait_event(after)
+            with torch.cuda.stream(stream):
+                dout, dpout = dbuf[k % 2][4:]
+                if hs.B:
+                    hout[:hs.B].copy_(dout[:hs.B], non_blocking=True)
+                if n_pf(hs):
+                    hpout[:hs.n_prefill].copy_(dpout[:hs.n_prefill], non_blocking=True)
+                read[k].record(stream)
+            nbytes["d2h"] += hs.B * Hq * D * 2 + n_pf(hs)
+
+        for stream in (cs_in, cs_out):  # first use of each copy stream, untimed
+            with torch.cuda.stream(stream):
+                dmeta[0][:16].copy_(hsteps[0].packed[:16], non_blocking=True)
         torch.cuda.synchronize()
         # as in the device-timed legs, the stream is held while the host
-        # enqueues every step (a serving loop runs its host work ahead of the
-        # GPU); each step's events still cover its own host->device copies,
-        # the step and the device->host read of its outputs
-        torch.cuda._sleep(hold_cycles(len(hsteps)))
-        for hs, (e0, e1) in zip(hsteps, ee):
+        # enqueues every step (a serving loop runs its host work ahead of the GPU)
+        torch.cuda._sleep(hold_cycles(n))
+        for k in range(n):
             flush()
+            e0, e1 = ee[k]
             e0.record(st)
-            ds = hs.to(device)
-            nq, nt = hs.B * Hq * D * 2, hs.T * Hkv * D * 2
-            npf = hs.n_prefill * Hq * D * 2 if attend_prefill else 0
-            if hs.B:
-                dq[:hs.B].copy_(hq[:hs.B], non_blocking=True)
-            if hs.T:
-                dk[:hs.T].copy_(hk[:hs.T], non_blocking=True)
-                dv[:hs.T].copy_(hv[:hs.T], non_blocking=True)
-            if npf:
-                dpq[:hs.n_prefill].copy_(hpq[:hs.n_prefill], non_blocking=True)
-            ex.enqueue(ds, dq, out, dk, dv, dpq, pout)
-            if hs.B:
-                hout[:hs.B].copy_(out[:hs.B], non_blocking=True)
-            if npf:
-                hpout[:hs.n_prefill].copy_(pout[:hs.n_prefill], non_blocking=True)
+            if k == 0:
+                bring_in(0, e0)
+            if k + 1 < n:
+                bring_in(k + 1, e0)  # into the other buffer set, free since step k-1 ended
+            if k > 0:
+                read_back(k - 1, cs_out, e0)  # step k-1's outputs, done before step k began
+            st.wait_event(landed[k])
+            dq, dk, dv, dpq, dout, dpout = dbuf[k % 2]
+            ex.enqueue(dsteps_e2e[k], dq, dout, dk, dv, dpq, dpout)
+            ran[k].record(st)
+            if k + 1 == n:
+                read_back(k, st, ran[k])
+            for ev in ([landed[k + 1]] if k + 1 < n else []) + ([read[k - 1]] if k > 0 else []):
+                st.wait_event(ev)
             e1.record(st)
-            h2d += hs.nbytes() + nq + 2 * nt + npf
-            d2h += nq + npf
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
-        e2e = {"ms": e2e_ms, "h2d": h2d / len(hsteps), "d2h": d2h / len(hsteps), "kvb": kvb}
+        e2e_steps = [a.elapsed_time(b) for a, b in ee]
+        e2e = {"ms": sum(e2e_steps), "h2d": nbytes["h2d"] / n, "d2h": nbytes["d2h"] / n, "kvb": kvb,
+               "step_ms": e2e_steps}
 
     return dict(tot_ms=tot_ms, step_ms=step_ms, dec_ms=dec_ms, kvb=kvb, seqsteps=seqsteps, algb=algb, algf=algf,
                 launches=launches, clocks=clk.summary(), e2e=e2e, plan_ms=t_plan * 1e3, tr=tr, plans=plans,
@@ -729,10 +775,14 @@ def main():
             line["e2e"] = {"value": e["kvb"] / (e["ms"] / 1e3) / 1e9, "unit": "GB/s",
                            "h2d_bytes_per_step": int(e["h2d"]), "d2h_bytes_per_step": int(e["d2h"]),
                            "ms_per_step": e["ms"] / args.steps,
-                           "timing": "per step: pinned host->device copies of the step's metadata, q and new "
-                                     "K/V, the step through the C ABI, device->host read of its outputs, all "
-                                     "inside the step's CUDA events; host enqueue runs ahead of the GPU; L2 "
-                                     "flushed between steps outside the events"}
+                           "ms_per_step_min_median_max": [min(e["step_ms"]), statistics.median(e["step_ms"]),
+                                                          max(e["step_ms"])],
+                           "timing": "per step, inside its CUDA events: the step through the C ABI and, on "
+                                     "two copy streams overlapping it, the pinned host->device copy of the next "
+                                     "step's metadata, q and new K/V and the device->host read of the previous "
+                                     "step's outputs (step 0 also copies its own inputs, the last step reads its "
+                                     "own outputs); host enqueue runs ahead of the GPU; L2 flushed between steps "
+                                     "outside the events"}
         pf = r.get("prefill") or leg
         if pf:
             line["prefill"] = prefill_block(pf)

@@ -83,12 +83,17 @@ class DeviceStep:
         self.max_chunk = plan.max_chunk
         self.pb = cascade_blocks(plan, cascade)  # 0: plain decode
 
-    def to(self, device, non_blocking=True):
-        """Device copy of a packed step: one host-to-device copy, then views."""
+    def to(self, device, non_blocking=True, out=None):
+        """Device copy of a packed step: one host-to-device copy (into `out`,
+        a uint8 device tensor of at least ``nbytes()``, if given), then views."""
         import torch
         d = object.__new__(DeviceStep)
         d.__dict__.update(self.__dict__)
-        buf = self.packed.to(device, non_blocking=non_blocking)
+        if out is None:
+            buf = self.packed.to(device, non_blocking=non_blocking)
+        else:
+            buf = out[:self.packed.numel()]
+            buf.copy_(self.packed, non_blocking=non_blocking)
         tdt = {np.int32: torch.int32, np.int64: torch.int64}
         for k, dt, o, shape in self.layout:
             n = int(np.prod(shape)) * np.dtype(dt).itemsize
