@@ -6,7 +6,11 @@
 //           (the prefill kernel's K/V loads);
 //   mode 1: 1-D bulk copies of a block's 4 KB;
 //   mode 2: 1-D bulk copies of 2 KB;
-//   LSU:    16-byte cp.async from 128 threads.
+//   LSU:    16-byte cp.async from 128 threads;
+//   pair:   clusters of 2 CTAs walking the same tiles, each loading the whole
+//           tile by TMA (pair mode 0), or loading half by TMA and pushing it
+//           into the other CTA's slot with a shared::cta -> shared::cluster
+//           bulk copy (pair mode 1).
 // Prints bytes per clock per SM.  Every wait is bounded (2 s), every copy
 // stays inside its buffer and its ring slot.
 // Build and run: nvcc -gencode arch=compute_100a,code=sm_100a -O3 -std=c++17
@@ -107,6 +111,116 @@ __global__ void __launch_bounds__(128, 1) bench_lsu(const uint8_t *base, int nbl
     if (tid == 0) out[blockIdx.x] = t1 - t0;
 }
 
+constexpr int HALF = 16384;
+
+__device__ __forceinline__ uint32_t cluster_rank() { uint32_t r; asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r)); return r; }
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
+    uint32_t r; asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank)); return r;
+}
+__device__ __forceinline__ void remote_arrive(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+__device__ __forceinline__ void push_to_peer(uint32_t dst_remote, const void *src, uint32_t bytes, uint32_t remote_bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst_remote),
+                 "r"(smem_addr(src)), "r"(bytes), "r"(remote_bar) : "memory");
+}
+
+// mode 0: whole tile by TMA (16 boxes) per CTA; mode 1: half by TMA + push of the half to the peer
+__global__ void __launch_bounds__(32, 1) bench_pair(const __grid_constant__ CUtensorMap tm, int nblk, int S, int mode, int iters,
+                                               long long *out, unsigned *err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * TILE);  // [S]: own half (arrive) + pushed half (tx) / whole tile
+    uint64_t *mine = full + S;                                       // [S]: own TMA half landed
+    uint64_t *pfree = mine + S;                                      // [S]: the peer's slot is free for my push
+    const int lane = threadIdx.x;
+    const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+    if (lane == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], mode ? 2 : 1);
+            mbar_init(&mine[i], 1);
+            mbar_init(&pfree[i], 1);
+        }
+        fence_mbar_init();
+    }
+    __syncwarp();
+    cluster_sync();  // barriers of both CTAs initialised before any remote access
+    const uint64_t dl = wait_deadline();
+    uint32_t seed = (blockIdx.x >> 1) * 7919u + 17u;  // both CTAs of a pair walk the same tiles
+    long long t0 = clock64();
+    bool ok = true;
+    int issued = 0;
+    for (int it = 0; it < iters && ok; ++it) {
+        const int s = it % S, use = it / S;
+        // the slot's previous tile: consumed (here: landed) before it is refilled
+        if (use > 0) ok = mbar_wait(&full[s], (use - 1) & 1, dl);
+        if (!ok) break;
+        if (mode == 1) {
+            if (lane == 0) remote_arrive(map_peer(smem_addr(&pfree[s]), peer));  // my slot s is free for the peer
+            // the peer's slot s is free for my push; the peer signals use u only once its slot's
+            // previous tile (with my previous push) has landed, so my previous push has also
+            // finished reading my slot before my TMA below overwrites it
+            ok = mbar_wait(&pfree[s], use & 1, dl);
+            if (!ok) break;
+        }
+        issued = it + 1;
+        seed = seed * 1664525u + 1013904223u;
+        uint8_t *slot = smem + s * TILE;
+        if (mode == 0) {
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], TILE);
+            __syncwarp();
+            if (lane < 8) {
+                const int blk = (int)(((seed >> 8) + (unsigned)lane * 2654435761u) % (unsigned)nblk);
+                tma_load_2d(slot + lane * 2048, &tm, 0, blk * 16, &full[s]);
+                tma_load_2d(slot + 16384 + lane * 2048, &tm, 64, blk * 16, &full[s]);
+            }
+            __syncwarp();
+        } else {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[s], HALF);   // the peer's pushed half
+                mbar_arrive_expect_tx(&mine[s], HALF);   // my own half
+            }
+            __syncwarp();
+            if (lane < 4) {  // blocks 4*rank + lane of the tile, both atom columns
+                const int b = 4 * (int)rank + lane;
+                const int blk = (int)(((seed >> 8) + (unsigned)b * 2654435761u) % (unsigned)nblk);
+                tma_load_2d(slot + b * 2048, &tm, 0, blk * 16, &mine[s]);
+                tma_load_2d(slot + 16384 + b * 2048, &tm, 64, blk * 16, &mine[s]);
+            }
+            __syncwarp();
+            ok = mbar_wait(&mine[s], use & 1, dl);
+            if (!ok) break;
+            if (lane == 0) {
+                const uint32_t rb = map_peer(smem_addr(&full[s]), peer);
+                for (int at = 0; at < 2; ++at) {
+                    uint8_t *src = slot + at * 16384 + rank * 8192;  // my 4 blocks of atom column at
+                    push_to_peer(map_peer(smem_addr(src), peer), src, 8192, rb);
+                }
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                mbar_arrive(&full[s]);  // my own half is in place
+            }
+            __syncwarp();
+        }
+    }
+    // drain: the last fill of every slot, my pushes' reads
+    const uint64_t dd = ok ? dl : drain_deadline();
+    for (int s = 0; s < S && s < issued; ++s) {
+        const int last = s + S * ((issued - 1 - s) / S);
+        if (!mbar_wait(&full[s], (last / S) & 1, dd)) ok = false;
+    }
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    long long t1 = clock64();
+    __syncwarp();
+    cluster_sync();  // no CTA leaves while the peer may still write into it
+    if (lane == 0) {
+        out[blockIdx.x] = t1 - t0;
+        if (!ok) atomicOr(err, 1u);
+    }
+}
+
 int main() {
     const int nblk = 16384;  // 64 MB of 4 KB blocks (L2-sized working set: 126 MB L2)
     const size_t bytes = (size_t)nblk * 4096;
@@ -162,5 +276,33 @@ int main() {
         printf("mode LSU cp.async 16 B, 128 threads, groups in flight %d: %.1f B/clk per SM, %.2f TB/s\n", S == 1 ? 1 : (S == 2 ? 2 : 4), bpc,
                bpc * sms * 1.965e9 / 1e12);
     }
+    // pairs of CTAs (clusters of 2) sharing each tile: mode 0 both load it whole by TMA, mode 1 each
+    // loads half by TMA and pushes that half into the other's slot (shared::cta -> shared::cluster)
+    const int grid = sms & ~1;
+    cudaFuncSetAttribute(bench_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    for (int mode = 0; mode < 2; ++mode)
+        for (int S : {2, 4}) {
+            const int sm = S * TILE + 3 * S * 8 + 1024 + 64;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(grid); cfg.blockDim = dim3(32); cfg.dynamicSmemBytes = sm;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2; attr[0].val.clusterDim.y = 1; attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr; cfg.numAttrs = 1;
+            for (int rep = 0; rep < 2; ++rep) {
+                cudaError_t e = cudaLaunchKernelEx(&cfg, bench_pair, tm, nblk, S, mode, iters, out, err);
+                if (e != cudaSuccess) { printf("launch error %s\n", cudaGetErrorString(e)); return 1; }
+                e = cudaDeviceSynchronize();
+                if (e != cudaSuccess) { printf("cuda error %s\n", cudaGetErrorString(e)); return 1; }
+            }
+            std::vector<long long> h(grid);
+            cudaMemcpy(h.data(), out, grid * sizeof(long long), cudaMemcpyDeviceToHost);
+            unsigned he = 0; cudaMemcpy(&he, err, 4, cudaMemcpyDeviceToHost);
+            double sum = 0;
+            for (auto v : h) sum += v;
+            const double bpc = (double)iters * TILE / (sum / grid);
+            printf("pair mode %d (%s) slots %d: %.1f B/clk per SM of tile data, err %u\n", mode,
+                   mode == 0 ? "whole tile by TMA" : "half by TMA + half pushed by the peer", S, bpc, he);
+        }
     return 0;
 }
