@@ -16,24 +16,27 @@
 //    (chunk, kv head) that share every K/V tile.
 //  * Warp roles: warps 0-7 and 8-15 are the softmax warpgroups of query
 //    tiles 0 and 1 (two threads per accumulator row = TMEM lane, each with
-//    half of the row's keys and of its O columns); warp 16 gathers
-//    K/V tiles of 128 keys (8 paged blocks) through the block table with
-//    2-D TMA tensor copies (64-column boxes, 128-byte swizzle, no multicast)
-//    into a ring of K and V slots; one lane of warp 17 issues the tcgen05
-//    MMAs (kind::f16, bf16 in, fp32 accumulate) and commits them to
+//    half of the row's keys and of its O columns); warp 16 gathers K/V
+//    tiles of 128 keys (8 paged blocks) through the block table with 2-D
+//    TMA tensor copies (64-column boxes, 128-byte swizzle, no multicast)
+//    into rings of K and V slots (an E4M3 cache: warps 16-17 gather the
+//    codes and widen them to f16); one lane of the last warp issues the
+//    tcgen05 MMAs (kind::f16, fp32 accumulate) and commits them to
 //    mbarriers.
 //  * Per K/V tile j and query tile t: S_t = Q_t K_j^T into TMEM; softmax
-//    warpgroup t reads S_t, writes P_t as bf16 into the first half of the
-//    same TMEM columns, and O_t += P_t V_j reads P_t straight from TMEM (the
-//    A operand of the MMA), so P never goes through shared memory and the
-//    tensor core's shared-memory reads are only Q, K and V.  The two query
-//    tiles alternate: the tensor core works on one tile's products while
-//    the other tile's softmax runs.
-//  * S_t(j+1) is issued only after O_t += P_t(j) V_j has completed (it
-//    overwrites P_t), so when softmax t sees S_t(j+1) the previous P.V is
-//    done and a rescale of its O row in TMEM is safe.  The MMA warp issues,
-//    per tile in turn, P.V as soon as P arrives and then the tile's next S,
-//    so a tile never waits for the other tile's softmax.
+//    warpgroup t loads S_t, computes P_t and hands it to O_t += P_t V_j.
+//  * bf16 cache: P_t goes to shared memory (128-byte swizzled, the A operand
+//    of the P.V MMA), so S_t(j+1) is issued into S_t's TMEM columns as soon
+//    as softmax t has loaded S_t(j) ("S free") and the tensor core computes
+//    the next scores while the exponentials run; softmax t writes P_t(j)
+//    once P_t(j-1).V has completed, which also makes a rescale of its O row
+//    in TMEM safe.  K_{j+1} is requested a tile period ahead (2 K slots),
+//    V_j once P(j-1).V is done (1 V slot).
+//  * E4M3 cache: P_t (f16) is written over the first half of S_t's TMEM
+//    columns and O_t += P_t V_j reads it from TMEM; S_t(j+1) is issued only
+//    after that P.V has completed.  The MMA warp issues, per tile in turn,
+//    P.V as soon as P arrives and then the tile's next S, so a tile never
+//    waits for the other tile's softmax.
 //  * Softmax applies the causal mask only on tiles that reach past the
 //    row's position, moves the running max only when it grows by more than
 //    8 (log2 units), and computes P with one packed FMA and one
