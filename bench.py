@@ -725,6 +725,11 @@ def main():
         leg = run_ours(largs, rank, world, device, workload="mixed", legs_only=True)["prefill"]
 
     tot_s, kvb, seqsteps = aggregate(r["tot_ms"] / 1e3, r["kvb"], r["seqsteps"], world, device)
+    e2e = r["e2e"]
+    if e2e is not None:  # whole job too: the slowest rank's time, every rank's bytes
+        e2e_s, e2e_kvb, e2e_h2d = aggregate(e2e["ms"] / 1e3, e2e["kvb"], e2e["h2d"], world, device)
+        _, _, e2e_d2h = aggregate(0.0, 0.0, e2e["d2h"], world, device)
+        e2e = dict(e2e, ms=e2e_s * 1e3, kvb=e2e_kvb, h2d=e2e_h2d, d2h=e2e_d2h)
 
     if rank == 0:
         peak, peak_kind = peaks()
@@ -772,8 +777,8 @@ def main():
             "blocks_copied_per_step": r.get("copies", 0) / args.steps,
             "preemptions": tr.sched.num_preemptions,
         }
-        if r["e2e"] is not None:
-            e = r["e2e"]
+        if e2e is not None:
+            e = e2e
             line["e2e"] = {"value": e["kvb"] / (e["ms"] / 1e3) / 1e9, "unit": "GB/s",
                            "h2d_bytes_per_step": int(e["h2d"]), "d2h_bytes_per_step": int(e["d2h"]),
                            "ms_per_step": e["ms"] / args.steps,
