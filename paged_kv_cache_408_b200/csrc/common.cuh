@@ -123,6 +123,13 @@ PA_DEVICE void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrive on named barrier `id` without waiting for it (the other threads of
+// the count wait with named_bar_sync).  A thread must not arrive on the same
+// barrier again before that phase completes.
+PA_DEVICE void named_bar_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ----------------------------------------------------------------- arithmetic
 // Packed fp32x2 fused multiply-add (sm_100): d = a * b + c, lane-wise, RN.
 PA_DEVICE float2 ffma2(float2 a, float2 b, float2 c) {

@@ -23,6 +23,13 @@
 //    codes and widen them to f16); one lane of the last warp issues the
 //    tcgen05 MMAs (kind::f16, fp32 accumulate) and commits them to
 //    mbarriers.
+//  * Start-up: the first loader thread initialises the barriers, requests
+//    the two query tiles (bf16: one 3-D TMA box per 64-column atom, 64
+//    columns x G heads x 128/G positions of q) and goes straight on to the
+//    block table and the first K tile, without waiting for the other
+//    warps, so the query tiles, the table entries and the first K tile are
+//    in flight together.  (An E4M3 cache's query rows are loaded and scaled
+//    by the softmax warps.)
 //  * Per K/V tile j and query tile t: S_t = Q_t K_j^T into TMEM; softmax
 //    warpgroup t loads S_t, computes P_t and hands it to O_t += P_t V_j.
 //  * bf16 cache: P_t goes to shared memory (128-byte swizzled, the A operand
@@ -63,6 +70,9 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;
+// Named barrier that releases the CTA once the barriers are initialised and
+// TMEM is allocated (the softmax warps' barriers use ids 1..4*NQ).
+constexpr int kStartBar = 15;
 // Of every 8 pairs of scores a softmax thread exponentiates, kEmuPairs go
 // through the FMA-pipe exponential (fastexp.cuh) and the rest through MUFU:
 // with head_dim 128 MUFU alone needs as many clocks per tile as the two
@@ -126,8 +136,8 @@ struct PCfg {
     static constexpr int X_BYTES = PSMEM ? 2 * NQ * NSPLIT * 128 * 2 : 3 * NQ * NSPLIT * 128 * 4;
     static constexpr int OFF_BAR = OFF_X + X_BYTES;
     // K/V full+empty; S full, P full, O done, O final; (P in shared memory)
-    // S free; end; (E4M3) K/V codes loaded
-    static constexpr int NBAR = 2 * NSK + 2 * NSV + 4 * NQ + (PSMEM ? NQ : 0) + 1 + (FP8 ? NSK + NSV : 0);
+    // S free; end; (E4M3) K/V codes loaded; (bf16) query tiles loaded
+    static constexpr int NBAR = 2 * NSK + 2 * NSV + 4 * NQ + (PSMEM ? NQ : 0) + 1 + (FP8 ? NSK + NSV : 1);
     static constexpr int USED = OFF_BAR + NBAR * 8 + 16;  // + the TMEM address slot
     // the tiles need a 1024-byte aligned base: slack to align it where the
     // budget allows, else the launch requires the base aligned (it is: the
@@ -156,7 +166,8 @@ struct PCfg {
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
-    prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+    prefill_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmQ) {
     constexpr int D = C::D, G = C::G, KT = C::KT, NSK = C::NSK, NSV = C::NSV, NQ = C::NQ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -170,6 +181,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     uint64_t *sfree = ofinal + NQ;                       // P in shared memory: S_t has been read
     uint64_t *mma_done = sfree + (C::PSMEM ? NQ : 0);
     uint64_t *kload = mma_done + 1, *vload = kload + NSK;  // E4M3: the codes of a tile have landed
+    uint64_t *qfull = mma_done + 1;                        // bf16: both query tiles have landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
     // [3][NQ][NSPLIT][128] fp32: max (2 parities), sum; with P in shared
     // memory [2][NQ][NSPLIT][128] bf16 maxima
@@ -232,7 +244,12 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
 
     if (w == C::W_MMA) tmem_alloc(tmem_slot, C::TMEM_COLS);
-    if (tid == 0) {
+    // The first loader thread sets up the barriers, requests the query tiles
+    // (bf16) and goes on to the K/V copies without waiting for the other
+    // warps (it arrives on the start barrier, they wait there), so the query
+    // tiles, the first block-table entries and the first K tile are all in
+    // flight at once.
+    if (tid == C::W_LOAD * 32) {
         for (int i = 0; i < NSK; ++i) {
             mbar_init(&kfull[i], C::FULL_ARRIVALS);
             mbar_init(&kempty[i], 1);
@@ -251,15 +268,30 @@ __global__ void __launch_bounds__(C::NT, 1)
         mbar_init(mma_done, 1);
         if constexpr (C::FP8)
             for (int i = 0; i < NSK + NSV; ++i) mbar_init(&kload[i], 1);
+        else
+            mbar_init(qfull, 1);
         fence_mbar_init();
+        if constexpr (!C::FP8) {
+            // ---- query tiles (bf16): row r of tile t = (position r / G,
+            // head r % G) is one 3-D box per 64-column atom (64 columns x G
+            // heads x QPOS positions of q, 128-byte swizzle).  Rows past the
+            // chunk are read as they stand (zeros past the end of q); they
+            // produce rows that are never stored.
+            mbar_arrive_expect_tx(qfull, NQ * C::QTILE);
+#pragma unroll
+            for (int t = 0; t < NQ; ++t)
+#pragma unroll
+                for (int at = 0; at < C::NATOM; ++at)
+                    tma_load_3d(sQ + t * C::QTILE + at * C::QATOM, &tmQ, at * 64, kvh * G, q_start + i0 + t * C::QPOS,
+                                qfull);
+        }
     }
-    // ---- query tiles: row r of tile t = (position r / G, head r % G), 128-byte swizzle.
-    // With an E4M3 cache the operands are f16: each row is scaled by a power
-    // of two 2^qexp that puts its largest magnitude in [2^14, 2^15) (exact for
-    // every bf16 value in f16's normal range), and 2^-qexp is folded into the
-    // row's softmax scale.
+    // ---- query tiles (E4M3 cache), by the softmax warps: the operands are
+    // f16, so each row is scaled by a power of two 2^qexp that puts its
+    // largest magnitude in [2^14, 2^15) (exact for every bf16 value in f16's
+    // normal range), and 2^-qexp is folded into the row's softmax scale.
     int qexp = 0;
-    if (w < C::NSMW) {
+    if (C::FP8 && w < C::NSMW) {
         const int t = w / (4 * C::NSPLIT), half = (w / 4) % C::NSPLIT, r = (w % 4) * 32 + lane;
         const int ip = i0 + t * C::QPOS + r / G;
         const bool valid = ip < clen;
@@ -308,11 +340,17 @@ __global__ void __launch_bounds__(C::NT, 1)
             *reinterpret_cast<uint4 *>(dst + at * C::QATOM + ((cc ^ (r & 7)) * 16)) = v[k];
         }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    uint32_t tmem = 0;
+    if (w == C::W_LOAD) {
+        __syncwarp();
+        named_bar_arrive(kStartBar, C::NT);
+    } else {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(kStartBar, C::NT);
+        tc_fence_after();
+        tmem = *tmem_slot;
+    }
     // ok turns false at the first wait that runs past the deadline; after
     // that no role issues another wait of the protocol: the loader and the
     // MMA warp stop issuing, the softmax warps only keep their named
@@ -499,6 +537,10 @@ __global__ void __launch_bounds__(C::NT, 1)
                 if (vissued > sl) mbar_wait(&vfull[sl], ((vissued - 1 - sl) / NSV) & 1, dd);
             __syncwarp();
         }
+        // the query tiles' copy has landed before the CTA may exit (the MMA
+        // warp waits for it before the first scores unless it gave up first)
+        if (!mbar_wait(qfull, 0, ok ? deadline : drain_deadline())) ok = false;
+        __syncwarp();
     } else if (w == C::W_MMA) {
         constexpr uint32_t idS = idesc_f16kind_f32(128, KT, false, !C::FP8);
         constexpr uint32_t idO = idesc_f16kind_f32(128, D, true, !C::FP8);
@@ -527,7 +569,7 @@ __global__ void __launch_bounds__(C::NT, 1)
                 __syncwarp();
             }
         };
-        if (ntiles > 0 && wait(&kfull[0], 0)) {
+        if (ntiles > 0 && (C::FP8 || wait(qfull, 0)) && wait(&kfull[0], 0)) {
 #pragma unroll
             for (int t = 0; t < NQ; ++t)
                 if (ntl[t] > 0) issue_s(t, 0);
@@ -908,6 +950,21 @@ bool code_map(CUtensorMap *map, const void *base, int64_t rows, int D) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// q [total_q][Hq][D] bf16 seen as a 3-D tensor (D, Hq, total_q); a box is
+// 64 columns x G heads x 128/G positions = the 128 rows of one atom column
+// of a query tile (row = position * G + head), 128-byte swizzled.
+bool query_map(CUtensorMap *map, const void *base, int total_q, int Hq, int D, int G) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)total_q};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(128 / G)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <class C>
 cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
     static std::mutex mu;
@@ -924,13 +981,15 @@ cudaError_t run_prefill(const PrefillArgs &a, cudaStream_t st) {
             ready[dev] = true;
         }
     }
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, tq = {};
     const int64_t rows = a.num_blocks * a.Hkv * 16;
     auto map = C::FP8 ? code_map : cache_map;
     if (!map(&tk, a.k_cache, rows, C::D) || !map(&tv, a.v_cache, rows, C::D)) return cudaErrorInvalidValue;
+    // (an E4M3 cache takes the query rows through registers, to scale them)
+    if (!C::FP8 && !query_map(&tq, a.q, a.total_q, a.Hq, C::D, C::G)) return cudaErrorInvalidValue;
     dim3 grid((a.max_q_len + C::NQ * C::QPOS - 1) / (C::NQ * C::QPOS), a.Hkv,
               a.shared_len > 0 ? std::max(a.key_splits, 1) : a.n_chunks);
-    return launch_pdl(prefill_kernel<C>, grid, dim3(C::NT), C::SMEM, st, a, tk, tv);
+    return launch_pdl(prefill_kernel<C>, grid, dim3(C::NT), C::SMEM, st, a, tk, tv, tq);
 }
 
 template <int D, bool FP8>

@@ -148,4 +148,13 @@ PA_DEVICE void tma_load_2d(void *dst_smem, const CUtensorMap *map, int c0, int c
         : "memory");
 }
 
+// 3-D tiled tensor copy global -> shared, completing on `bar`.  No multicast.
+PA_DEVICE void tma_load_3d(void *dst_smem, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_addr(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+        : "memory");
+}
+
 }  // namespace pa

@@ -206,10 +206,10 @@ def explore(ntl, nslot, seeds, skip_odd_odone=False, no_odone_wait=False, fp8=Fa
     return None
 
 
-def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
+def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False, skip_qwait=False):
     """Random schedules of the P-in-shared-memory protocol (a K ring of nsk
-    slots, a V ring of nsv slots, a P buffer per query tile); None or the
-    first violation."""
+    slots, a V ring of nsv slots, a P buffer per query tile, the query tiles
+    copied once by the loader thread); None or the first violation."""
     nq, ntiles = len(ntl), max(ntl)
     for seed in range(seeds):
         rnd = random.Random(7000 + seed)
@@ -221,7 +221,8 @@ def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
         s_data = [-1] * nq   # the key tile whose scores sit in S_t's TMEM columns
         p_data = [-1] * nq   # the key tile whose P sits in P_t's buffer
         pv_done = [-1] * nq
-        pending, violation = [], []
+        qbar, q_landed = Barrier("qfull"), [False]
+        pending, side, violation = [], [], []
 
         class Done:  # an asynchronous completion: apply its effect, then arrive
             def __init__(self, bar, effect=None):
@@ -246,12 +247,16 @@ def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
             pending.append(Done(ring[kind + "full"][sl], landed(kind, j)))
 
         def loader():
+            # the query tiles' copy completes on its own, in no order with
+            # the K/V copies and the MMAs (the side queue)
+            side.append(Done(qbar, lambda: q_landed.__setitem__(0, True)))
             if ntiles:
                 yield from fill("k", 0)
             for j in range(ntiles):
                 if j + 1 < ntiles:
                     yield from fill("k", j + 1)
                 yield from fill("v", j)
+            yield qbar, 0  # the copy has landed before the CTA may exit
 
         def consumed_by(kind, sl, j):
             def f():
@@ -260,6 +265,8 @@ def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
 
         def scores(t, j):
             def f():
+                if not q_landed[0]:
+                    violation.append(f"S_{t}({j}) computed before the query tiles landed")
                 if held["k"][j % nsk] != j:
                     violation.append(f"S_{t}({j}) computed from K tile {held['k'][j % nsk]}")
                 s_data[t] = j
@@ -276,6 +283,8 @@ def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
 
         def mma():
             if ntiles:
+                if not skip_qwait:
+                    yield qbar, 0
                 yield ring["kfull"][0], 0
                 for t in range(nq):
                     if ntl[t]:
@@ -323,24 +332,29 @@ def explore_psmem(ntl, nsk, nsv, seeds, skip_sfree=False, skip_odone=False):
                     yield None, f"epilogue of tile {t} before its last P.V"
 
         actors = {"load": loader(), "mma": mma(), **{f"softmax{t}": softmax(t) for t in range(nq)}}
-        err = run_schedule(actors, pending, rnd)
+        err = run_schedule(actors, pending, rnd, side)
         if err or violation:
             return f"seed {seed}: {err or violation[0]}"
     return None
 
 
-def run_schedule(actors, pending, rnd):
+def run_schedule(actors, pending, rnd, side=None):
     """Drive generator actors that yield (barrier, phase) waits, or (None,
     message) for a violation; completions in `pending` arrive in order at
     random times, and an actor that could run is delayed now and then (so a
     completion may overtake a thread between its wait and its next step).
-    Returns None or the first violation / deadlock."""
+    Completions in `side` arrive one at a time in any order and at any time
+    (another engine's).  Returns None or the first violation / deadlock."""
+    side = [] if side is None else side
     waiting = {k: None for k in actors}
     done = set()
     while len(done) < len(actors):
         progress = False
         if pending and rnd.random() < 0.5:
             pending.pop(0).arrive()
+            progress = True
+        if side and rnd.random() < 0.1:
+            side.pop(rnd.randrange(len(side))).arrive()
             progress = True
         order = list(actors)
         rnd.shuffle(order)
@@ -367,8 +381,8 @@ def run_schedule(actors, pending, rnd):
                 done.add(k)
             progress = True
         if not progress:
-            if pending:
-                pending.pop(0).arrive()
+            if pending or side:
+                (pending if pending and (not side or rnd.random() < 0.5) else side).pop(0).arrive()
                 continue
             stuck = {k: (w[0].name, w[1]) for k, w in waiting.items() if w and k not in done}
             return f"deadlock {stuck}"
@@ -397,6 +411,12 @@ def test_psmem_protocol_has_no_deadlock_stale_data_or_overwrite(ntl, nsk, nsv):
 def test_psmem_skipped_s_free_wait_is_caught():
     found = [explore_psmem([6, 7], 2, 1, seeds=200, skip_sfree=True),
              explore_psmem([9, 10], 3, 3, seeds=200, skip_sfree=True)]
+    assert all(found), found
+
+
+def test_psmem_scores_issued_before_the_query_tiles_landed_is_caught():
+    found = [explore_psmem([3, 4], 2, 1, seeds=200, skip_qwait=True),
+             explore_psmem([1, 0], 3, 3, seeds=200, skip_qwait=True)]
     assert all(found), found
 
 
@@ -460,6 +480,7 @@ def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_fail
         tile = {k: [Barrier(f"{k}{t}", 2 if k in ("pfull", "sfree") else 1) for t in range(nq)]
                 for k in ("sfull", "sfree", "pfull", "odone", "ofinal")}
         mma_done = Barrier("mma_done")
+        qbar = Barrier("qfull")
         pending = []
         drop_at = rnd.randrange(1, 4 * ntiles * (nq + 2) + 2)
         sent = [0]
@@ -568,6 +589,7 @@ def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_fail
                 post(ring[kind + "full"][sl])
                 return True
 
+            post(qbar)  # the query tiles (may be the completion that is lost)
             if ntiles:
                 ok = yield from fill("k", 0, ok)
             for j in range(ntiles):
@@ -583,10 +605,15 @@ def explore_give_up(ntl, nslot, seeds, break_softmax_loop=False, wait_after_fail
                     for sl in range(ns[kind]):
                         if issued[kind] > sl:
                             yield ("drain", ring[kind + "full"][sl], (issued[kind] - 1 - sl) // ns[kind])
+            # the query copy has landed before exit: on the launch's deadline,
+            # or after a failure on the short drain budget
+            r = yield ("wait" if ok else "drain", qbar, 0)
+            ok = ok and r
 
         def mma_ps():
             ok = True
             if ntiles:
+                ok = yield from wait(qbar, 0, ok)
                 ok = yield from wait(ring["kfull"][0], 0, ok)
                 if ok:
                     for t in range(nq):
