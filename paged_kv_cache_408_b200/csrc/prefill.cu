@@ -213,6 +213,16 @@ __global__ void __launch_bounds__(C::NT, 1)
     // causal chunk: rows are positions pfx + i, keys [0, pfx + i]; shared
     // prefix: rows are sequences, keys [0, shared_len) for every row
     const bool shared = a.shared_len > 0;
+    // a shared prefix is split over its keys (grid z): this CTA attends key
+    // tiles [jt0, jt1) and writes split-K piece blockIdx.z of its rows
+    const int ks = shared ? (int)gridDim.z : 1, kz = shared ? (int)blockIdx.z : 0;
+    const int jt0 = shared ? kz * ((a.shared_len + KT - 1) / KT) / ks : 0;
+    const int jt1 = shared ? (kz + 1) * ((a.shared_len + KT - 1) / KT) / ks : 0;
+    // the loader's first window of 32 block-table entries (lane l: entry
+    // jt0 * KT/16 + l), requested together with the chunk's lengths; entries
+    // past the sequence's last block are never used
+    const int32_t *bt = a.block_tables + (size_t)c * a.max_blocks;
+    const int went0 = w == C::W_LOAD ? bt[min(jt0 * (KT / 16) + lane, a.max_blocks - 1)] : 0;
     const int q_start = shared ? 0 : a.cu_q[c];
     const int clen = shared ? a.total_q : a.cu_q[c + 1] - q_start;
     const int pfx = shared ? a.shared_len : a.prefix_lens[c];
@@ -223,16 +233,10 @@ __global__ void __launch_bounds__(C::NT, 1)
         return;
     }
     const int nalloc = (L + 15) >> 4;  // blocks of the sequence
-    // a shared prefix is split over its keys (grid z): this CTA attends key
-    // tiles [jt0, jt1) and writes split-K piece blockIdx.z of its rows
-    const int ks = shared ? (int)gridDim.z : 1, kz = shared ? (int)blockIdx.z : 0;
-    const int jt0 = shared ? kz * ((L + KT - 1) / KT) / ks : 0;
-    const int jt1 = shared ? (kz + 1) * ((L + KT - 1) / KT) / ks : 0;
     if (shared && jt1 <= jt0) {  // more splits than key tiles
         if (tid == 0) flag_error(a.err, PA_DEVERR_BAD_LEN);
         return;
     }
-    const int32_t *bt = a.block_tables + (size_t)c * a.max_blocks;
     // K/V tiles each query tile needs (causal: up to its last valid row)
     int ntl[NQ], ntiles = 0;
 #pragma unroll
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         constexpr int NS = C::NSK;    // K and V slots (as many of each)
         const int ct = tid - C::W_LOAD * 32;
         const bool issuer = w == C::W_LOAD;
-        int win0 = jt0 * BPT, went = issuer ? bt[min(win0 + lane, nalloc - 1)] : 0;
+        int win0 = jt0 * BPT, went = went0;
         auto stage = [&](int s, int kv) -> uint8_t * {
             if constexpr (C::STG_IN_PLACE) return (kv ? sV : sK) + s * C::KTILE + C::KATOM;
             return smem + C::OFF_STG + (2 * s + kv) * C::STG_BYTES;
@@ -483,7 +487,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         // refilled every 32/BPT tiles, so a tile's copies are issued without
         // a global round trip; a tile's row is kept from its K copy for its V.
         constexpr int BPT = KT / 16;  // blocks per tile
-        int win0 = jt0 * BPT, went = bt[min(win0 + lane, nalloc - 1)];
+        int win0 = jt0 * BPT, went = went0;
         auto tile_row = [&](int jj) {  // lanes 0..BPT-1: cache row of block jj*BPT + lane (tiles in order)
             const int jb = (jt0 + jj) * BPT;
             if (jb + BPT > win0 + 32) {
