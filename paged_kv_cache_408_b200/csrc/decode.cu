@@ -1037,9 +1037,15 @@ __global__ void __launch_bounds__(C::NT, C::MIN_CTAS) decode_kernel(const Decode
 // piece; 2 in plain decode), so the look-ahead never reads a stale slot
 // (after an L2 flush, from DRAM).  The rest of a row's pieces are loaded
 // once its count is known.
+// Pieces a merge warp loads at a time (its first round trip holds at most
+// this many; a larger count is merged in further chunks).  4 keeps the
+// kernel at 47 registers, 40 warps an SM; with 8 it took 64 registers and
+// a 256-sequence cascade's 16,384-row merge ran ~1 us longer.
+constexpr int kMergeFirst = 4;
+
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
-    constexpr int E = D / 32, kFirst = 8;
+    constexpr int E = D / 32, kFirst = kMergeFirst;
     pdl_trigger();
     pdl_wait();
     const int lane = threadIdx.x & 31;
@@ -1168,7 +1174,7 @@ cudaError_t run(const DecodeArgs &a, cudaStream_t st) {
     // pieces every merged row is sure to have: a cascade row has its prefix
     // pieces and (unless its suffix is empty) one suffix piece; a plain row
     // that needs a merge has at least two
-    m.merge_spec = std::min({8, a.max_parts, a.prefix_blocks ? a.prefix_pieces + 1 : 2});
+    m.merge_spec = std::min({kMergeFirst, a.max_parts, a.prefix_blocks ? a.prefix_pieces + 1 : 2});
     return launch_pdl(merge_kernel<C::D>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, st, m);
 }
 
